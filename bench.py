@@ -1,0 +1,402 @@
+"""Benchmark of the HISA hot path on B200.
+
+One step = one pass of the whole path over the 64K prefill workload: the
+indexer (block sums, block selection, token selection) followed by sparse
+MQA attention, L=65536, B=128, m=64, k=2048, d_idx=d=128, H=64, seed 0.
+`value` is prefill tokens/s (queries processed per second, all ranks).
+The decode half of the metric (batch 32 at context 131072, one query per
+sequence per step) is measured in the same run and reported under "decode".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl hsa|reference]
+
+--impl reference times the CPU oracle on a bounded sample of the same
+workload (host cores; rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "prefill tokens/s at 64K and decode queries/s at 128K (index + sparse attn)"
+PREFILL = synth.WORKLOADS["prefill_64k"]
+DECODE = synth.WORKLOADS["decode_128k_b32"]
+L2_FLUSH_BYTES = 512 << 20
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained", d["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu: int):
+        self.gpu, self.proc, self.lines = gpu, None, []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- helpers
+
+_INPUTS = {}
+
+
+def prefill_inputs():
+    if "prefill" not in _INPUTS:
+        _INPUTS["prefill"] = synth.prefill_inputs(PREFILL)
+    return _INPUTS["prefill"]
+
+
+def dev_bf16(u16, device):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(u16).view(np.int16)).to(device).view(torch.bfloat16)
+
+
+def pinned_bf16(u16):
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(u16).view(np.int16)).view(torch.bfloat16)
+    return t.pin_memory()
+
+
+def attn_flops(idx_counts, H, d):
+    # QK^T and PV: 2 * 2 * H * d multiply-adds per kept (query, key) pair
+    return 4.0 * H * d * float(idx_counts)
+
+
+# ---------------------------------------------------------------- our arm
+
+def bench_hsa(args, rank, world, device):
+    import torch
+    import hierarchical_sparse_attention_hisa_b200 as hsa
+
+    hsa.load()
+    w = PREFILL
+    x = prefill_inputs()
+    q_idx, k_idx = dev_bf16(x["q_idx"], device), dev_bf16(x["k_idx"], device)
+    Q, K, V = dev_bf16(x["Q"], device), dev_bf16(x["K"], device), dev_bf16(x["V"], device)
+    p = hsa.params(B=w.B, m=w.m, k=w.k, d_idx=w.d_idx, H=w.H, d=w.d)
+    ws = torch.empty(hsa.hsa_index_workspace_size(p, w.Lq, w.L), dtype=torch.uint8, device=device)
+    idx = torch.empty((w.Lq, w.k), dtype=torch.int32, device=device)
+    O = torch.empty((w.Lq, w.H, w.d), dtype=torch.bfloat16, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        hsa.hsa_index(p, w.Lq, w.L, q_idx, k_idx, idx, ws, stream)
+        if ev:
+            ev[1].record(stream)
+        hsa.hsa_sparse_attn(p, w.Lq, w.L, Q, K, V, idx, O, stream)
+        if ev:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    kept = int((idx >= 0).sum().item())
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    launches0 = hsa.kernel_launches()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for s in range(args.steps):
+            flush.zero_()          # evict L2 between timed steps (outside the events)
+            step(evs[s])
+        torch.cuda.synchronize()
+    launches = hsa.kernel_launches() - launches0
+    if world > 1:
+        torch.distributed.barrier()
+    t_index = [e[0].elapsed_time(e[1]) for e in evs]
+    t_attn = [e[1].elapsed_time(e[2]) for e in evs]
+    ms_step = sum(a + b for a, b in zip(t_index, t_attn)) / args.steps
+    ms_step = max_over_ranks(ms_step, world, device)
+    attn_ms = sum(t_attn) / args.steps
+
+    # end to end through the public API: pinned host inputs -> device, result -> host
+    e2e = None
+    if not args.skip_e2e:
+        hq, hk = pinned_bf16(x["q_idx"]), pinned_bf16(x["k_idx"])
+        hQ, hK, hV = pinned_bf16(x["Q"]), pinned_bf16(x["K"]), pinned_bf16(x["V"])
+        hO = torch.empty(O.shape, dtype=torch.bfloat16).pin_memory()
+        hidx = torch.empty(idx.shape, dtype=torch.int32).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hQ, hK, hV))
+        d2h = hO.numel() * 2 + hidx.numel() * 4
+
+        def e2e_step():
+            for dst, src in ((q_idx, hq), (k_idx, hk), (Q, hQ), (K, hK), (V, hV)):
+                dst.copy_(src, non_blocking=True)
+            hsa.hsa_index(p, w.Lq, w.L, q_idx, k_idx, idx, ws, stream)
+            hsa.hsa_sparse_attn(p, w.Lq, w.L, Q, K, V, idx, O, stream)
+            hO.copy_(O, non_blocking=True)
+            hidx.copy_(idx, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        n_e2e = max(1, min(args.steps, 3))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms = max_over_ranks(a.elapsed_time(b) / n_e2e, world, device)
+        e2e = {"value": w.Lq * world / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h}
+        del hQ, hK, hV, hO
+
+    del Q, K, V, O, flush
+    torch.cuda.empty_cache()
+    dec = None if args.skip_decode else bench_decode(args, world, device)
+
+    hbm, tf, tf_sus, src = peaks()
+    flops = attn_flops(kept, w.H, w.d)
+    achieved = flops / (attn_ms / 1e3) / 1e12
+    res = {
+        "metric": METRIC,
+        "value": w.Lq * world / (ms_step / 1e3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "prefill_64k", "L": w.L, "Lq": w.Lq, "B": w.B, "m": w.m, "k": w.k,
+                   "d_idx": w.d_idx, "H": w.H, "d": w.d, "needles": w.needles, "batch": 1,
+                   "seq_len": w.L, "parallelism": f"replicas x{world}",
+                   "l2": "flushed (512 MiB write) between timed steps"},
+        "breakdown_ms": {"hsa_index": sum(t_index) / args.steps, "hsa_sparse_attn": attn_ms},
+        "roofline": {"kernel": "sparse attention", "bound": "tensor", "achieved": achieved,
+                     "peak": tf, "unit": "TFLOP/s", "frac": achieved / tf, "traffic": None,
+                     "peak_source": f"{src} bf16 burst",
+                     "flops_per_launch": flops},
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+        "e2e": e2e,
+        "decode": dec,
+    }
+    return res
+
+
+def bench_decode(args, world, device):
+    """Decode: batch 32 sequences at context 131072, one query each per step."""
+    import torch
+    import hierarchical_sparse_attention_hisa_b200 as hsa
+
+    w = DECODE
+    steps = max(1, min(args.decode_steps, w.decode_steps))
+    warm = min(args.warmup, 8)
+    cap = w.decode_ctx + warm + steps + w.B
+    cap = (cap + w.B - 1) // w.B * w.B
+    x = synth.decode_inputs(w, w.decode_ctx, cap, warm + steps)
+    p = hsa.params(B=w.B, m=w.m, k=w.k, d_idx=w.d_idx, H=w.H, d=w.d)
+    kc, Kc, Vc = (dev_bf16(x[n], device) for n in ("k_idx_cache", "K_cache", "V_cache"))
+    ksum = torch.zeros((w.batch, cap // w.B, w.d_idx), dtype=torch.float32, device=device)
+    for b in range(w.batch):
+        hsa.hsa_block_sums(p, w.decode_ctx, kc[b], ksum[b])
+    ctx = torch.full((w.batch,), w.decode_ctx, dtype=torch.int32, device=device)
+    new = {n: dev_bf16(x[n], device) for n in ("q_idx_new", "k_idx_new", "Q_new", "K_new", "V_new")}
+    ws = torch.empty(hsa.hsa_decode_workspace_size(p, w.batch, cap), dtype=torch.uint8, device=device)
+    O = torch.empty((w.batch, w.H, w.d), dtype=torch.bfloat16, device=device)
+    idx = torch.empty((w.batch, w.k), dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream()
+
+    def step(s):
+        hsa.hsa_decode_step(p, w.batch, cap, ctx, kc, Kc, Vc, ksum, new["q_idx_new"][s],
+                            new["k_idx_new"][s], new["Q_new"][s], new["K_new"][s], new["V_new"][s],
+                            O, idx, ws, stream)
+
+    for s in range(warm):
+        step(s)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for s in range(warm, warm + steps):
+        step(s)
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b) / steps, world, device)
+    hbm, _, _, src = peaks()
+    # algorithmic bytes per query: block sums read + kept blocks' index keys +
+    # kept K/V rows + Q and O rows
+    per_q = (w.decode_ctx // w.B) * w.d_idx * 4 + w.m * w.B * w.d_idx * 2 + w.k * w.d * 2 * 2 \
+        + 2 * w.H * w.d * 2
+    gbs = per_q * w.batch / (ms / 1e3) / 1e9
+    return {"metric": "decode queries/s at 128K", "value": w.batch * world / (ms / 1e3),
+            "unit": "queries/s", "ms_per_step": ms, "steps": steps, "batch": w.batch,
+            "ctx": w.decode_ctx, "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm,
+                                              "unit": "GB/s", "frac": gbs / hbm,
+                                              "peak_source": src,
+                                              "bytes_per_query": per_q}}
+
+
+def max_over_ranks(v, world, device):
+    if world <= 1:
+        return v
+    import torch
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- oracle arm
+
+def oracle_sample(target_s=15.0):
+    """Time the oracle (index + attention) on a bounded sample of query rows
+    of the 64K workload; returns (tokens/s, threads, description)."""
+    import oracle
+    w = PREFILL
+    x = prefill_inputs()
+    threads = oracle.default_threads()
+    rows = np.linspace(0, w.Lq - 1, 8 * threads).astype(np.int64)
+    t0 = time.perf_counter()
+    idx = oracle.index(x["q_idx"], x["k_idx"], w.B, w.m, w.k, rows=rows, threads=threads)
+    oracle.sparse_attn(x["Q"], x["K"], x["V"], idx, rows=rows, threads=threads)
+    dt = time.perf_counter() - t0
+    n = len(rows)
+    if dt < target_s:   # grow the sample towards the target duration
+        n = int(min(w.Lq, max(n, n * target_s / max(dt, 1e-3))))
+        rows = np.linspace(0, w.Lq - 1, n).astype(np.int64)
+        t0 = time.perf_counter()
+        idx = oracle.index(x["q_idx"], x["k_idx"], w.B, w.m, w.k, rows=rows, threads=threads)
+        oracle.sparse_attn(x["Q"], x["K"], x["V"], idx, rows=rows, threads=threads)
+        dt = time.perf_counter() - t0
+    return n / dt, threads, f"{n} evenly spaced query rows of the 64K prefill (index + attention), {dt:.1f} s"
+
+
+def bench_reference(args, rank, world):
+    if rank != 0:
+        return None
+    vals = []
+    desc = threads = None
+    for s in range(args.warmup + args.steps):
+        v, threads, desc = oracle_sample(target_s=float(os.environ.get("HSA_ORACLE_SECONDS", "10")))
+        if s >= args.warmup:
+            vals.append(v)
+    v = statistics.mean(vals)
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / v,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32/f64",
+            "data": "synthetic", "config": {"workload": "prefill_64k", "L": PREFILL.L,
+                                            "B": PREFILL.B, "m": PREFILL.m, "k": PREFILL.k,
+                                            "H": PREFILL.H, "d": PREFILL.d},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ---------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="hsa", choices=["hsa", "reference"])
+    ap.add_argument("--decode-steps", type=int, default=64)
+    ap.add_argument("--skip-decode", action="store_true")
+    ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--skip-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        res = bench_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    import torch
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    res = bench_hsa(args, rank, world, device)
+    if rank == 0 and world == 1 and not args.skip_cpu_baseline:
+        v, threads, desc = oracle_sample(target_s=float(os.environ.get("HSA_ORACLE_SECONDS", "15")))
+        res["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                               "sample": desc}
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

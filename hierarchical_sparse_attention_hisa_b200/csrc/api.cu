@@ -1,0 +1,246 @@
+// C ABI of libhsa.so (declared in include/hsa.h): host-side argument checks,
+// workspace layout and kernel launches. No allocation, no synchronisation.
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "hsa.h"
+#include "kernels.cuh"
+
+namespace hsa {
+static std::atomic<uint64_t> g_launches{0};
+void count_launches(int n) { g_launches.fetch_add(uint64_t(n), std::memory_order_relaxed); }
+}  // namespace hsa
+
+namespace {
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Candidates a selection stage keeps in shared memory per query.
+constexpr int64_t kMaxCandidates = 16384;
+
+int check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return HSA_ERR_CUDA;
+  static int cached_dev = -1, cached_ok = 0;
+  if (dev != cached_dev) {
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+      return HSA_ERR_CUDA;
+    cached_ok = major == 10;
+    cached_dev = dev;
+  }
+  return cached_ok ? HSA_OK : HSA_ERR_DEVICE;
+}
+
+int check_index_params(const hsa_params* p) {
+  if (!p) return HSA_ERR_ARG;
+  if (p->B < 1 || p->B > 1024) return HSA_ERR_ARG;
+  if (p->m < 2 || p->m > 256) return HSA_ERR_ARG;
+  if (p->k < 1 || p->k > 8192) return HSA_ERR_ARG;
+  if (p->d_idx != 64 && p->d_idx != 128) return HSA_ERR_ARG;
+  if (int64_t(p->m) * p->B > kMaxCandidates) return HSA_ERR_ARG;
+  return HSA_OK;
+}
+
+int check_attn_params(const hsa_params* p) {
+  if (!p) return HSA_ERR_ARG;
+  if (p->k < 1 || p->k > 8192) return HSA_ERR_ARG;
+  if (p->H < 1 || p->H > 128) return HSA_ERR_ARG;
+  if (p->d != 64 && p->d != 128) return HSA_ERR_ARG;
+  if (!(p->scale >= 0.f) || std::isinf(p->scale)) return HSA_ERR_ARG;
+  return HSA_OK;
+}
+
+float softmax_scale(const hsa_params* p) {
+  return p->scale > 0.f ? p->scale : 1.0f / std::sqrt(float(p->d));
+}
+
+int check_lengths(const hsa_params* p, int64_t Lq, int64_t Lk) {
+  if (Lq < 0 || Lk < 1 || Lq > Lk || Lq > (int64_t(1) << 31) - 1) return HSA_ERR_ARG;
+  if (Lk > (int64_t(1) << 31) - 1) return HSA_ERR_ARG;
+  if (Lk / p->B > kMaxCandidates) return HSA_ERR_ARG;
+  return HSA_OK;
+}
+
+int launch_status() {
+  return cudaGetLastError() == cudaSuccess ? HSA_OK : HSA_ERR_CUDA;
+}
+
+struct IndexWs {
+  size_t ksum_off, blocks_off, total;
+};
+IndexWs index_ws(const hsa_params* p, int64_t Lq, int64_t Lk) {
+  IndexWs w;
+  w.ksum_off = 0;
+  w.blocks_off = align_up(size_t(Lk / p->B) * p->d_idx * sizeof(float));
+  w.total = w.blocks_off + align_up(size_t(Lq) * p->m * sizeof(int32_t));
+  return w;
+}
+
+// Largest number of block candidates any query of [Lk-Lq, Lk) scores.
+int64_t max_block_candidates(const hsa_params* p, int64_t Lk) {
+  const int64_t nb = (Lk - 1) / p->B + 1;
+  return nb > 2 ? nb - 2 : 1;
+}
+
+}  // namespace
+
+extern "C" {
+
+uint64_t hsa_kernel_launches(void) { return hsa::g_launches.load(std::memory_order_relaxed); }
+
+const char* hsa_status_string(int status) {
+  switch (status) {
+    case HSA_OK: return "ok";
+    case HSA_ERR_ARG: return "invalid argument (null/misaligned pointer or unsupported size)";
+    case HSA_ERR_WORKSPACE: return "workspace missing or too small";
+    case HSA_ERR_CUDA: return "CUDA launch or runtime error";
+    case HSA_ERR_TIMEOUT: return "bounded device wait gave up";
+    case HSA_ERR_DEVICE: return "current device is not an sm_100 (B200-class) GPU";
+    default: return "unknown status";
+  }
+}
+
+int hsa_index_workspace_size(const hsa_params* p, int64_t Lq, int64_t Lk, size_t* bytes) {
+  if (!bytes) return HSA_ERR_ARG;
+  if (int e = check_index_params(p)) return e;
+  if (int e = check_lengths(p, Lq, Lk)) return e;
+  *bytes = index_ws(p, Lq, Lk).total;
+  return HSA_OK;
+}
+
+int hsa_block_sums(const hsa_params* p, int64_t Lk, const hsa_bf16* k_idx, float* ksum,
+                   cudaStream_t stream) {
+  if (int e = check_index_params(p)) return e;
+  if (Lk < 0) return HSA_ERR_ARG;
+  if (Lk / p->B == 0) return HSA_OK;
+  if (!aligned16(k_idx) || !aligned16(ksum)) return HSA_ERR_ARG;
+  if (int e = check_device()) return e;
+  hsa::launch_block_sums(k_idx, Lk, p->B, p->d_idx, ksum, stream);
+  return launch_status();
+}
+
+int hsa_select_blocks(const hsa_params* p, int64_t Lq, int64_t Lk, const hsa_bf16* q_idx,
+                      const float* ksum, int32_t* blocks, void* workspace,
+                      size_t workspace_bytes, cudaStream_t stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  if (int e = check_index_params(p)) return e;
+  if (int e = check_lengths(p, Lq, Lk)) return e;
+  if (Lq == 0) return HSA_OK;
+  if (!aligned16(q_idx) || !aligned16(blocks) || (Lk / p->B > 0 && !aligned16(ksum)))
+    return HSA_ERR_ARG;
+  if (int e = check_device()) return e;
+  hsa::RowMap rm{Lq, Lk, nullptr, 0};
+  hsa::launch_select_blocks(rm, Lq, q_idx, ksum, 0, p->B, p->m, p->d_idx, blocks,
+                            max_block_candidates(p, Lk), stream);
+  return launch_status();
+}
+
+int hsa_select_tokens(const hsa_params* p, int64_t Lq, int64_t Lk, const hsa_bf16* q_idx,
+                      const hsa_bf16* k_idx, const int32_t* blocks, int32_t* indices,
+                      void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  if (int e = check_index_params(p)) return e;
+  if (int e = check_lengths(p, Lq, Lk)) return e;
+  if (Lq == 0) return HSA_OK;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(blocks) || !aligned16(indices))
+    return HSA_ERR_ARG;
+  if (int e = check_device()) return e;
+  hsa::RowMap rm{Lq, Lk, nullptr, 0};
+  hsa::launch_select_tokens(rm, Lq, q_idx, k_idx, blocks, p->B, p->m, p->k, p->d_idx, indices,
+                            stream);
+  return launch_status();
+}
+
+int hsa_index(const hsa_params* p, int64_t Lq, int64_t Lk, const hsa_bf16* q_idx,
+              const hsa_bf16* k_idx, int32_t* indices, void* workspace, size_t workspace_bytes,
+              cudaStream_t stream) {
+  if (int e = check_index_params(p)) return e;
+  if (int e = check_lengths(p, Lq, Lk)) return e;
+  if (Lq == 0) return HSA_OK;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(indices)) return HSA_ERR_ARG;
+  const IndexWs w = index_ws(p, Lq, Lk);
+  if (!aligned16(workspace) || workspace_bytes < w.total) return HSA_ERR_WORKSPACE;
+  if (int e = check_device()) return e;
+  char* ws = static_cast<char*>(workspace);
+  float* ksum = reinterpret_cast<float*>(ws + w.ksum_off);
+  int32_t* blocks = reinterpret_cast<int32_t*>(ws + w.blocks_off);
+  hsa::launch_block_sums(k_idx, Lk, p->B, p->d_idx, ksum, stream);
+  hsa::RowMap rm{Lq, Lk, nullptr, 0};
+  hsa::launch_select_blocks(rm, Lq, q_idx, ksum, 0, p->B, p->m, p->d_idx, blocks,
+                            max_block_candidates(p, Lk), stream);
+  hsa::launch_select_tokens(rm, Lq, q_idx, k_idx, blocks, p->B, p->m, p->k, p->d_idx, indices,
+                            stream);
+  return launch_status();
+}
+
+int hsa_sparse_attn(const hsa_params* p, int64_t Lq, int64_t Lk, const hsa_bf16* Q,
+                    const hsa_bf16* K, const hsa_bf16* V, const int32_t* indices, hsa_bf16* O,
+                    cudaStream_t stream) {
+  if (int e = check_attn_params(p)) return e;
+  if (Lq < 0 || Lk < 1 || Lq > (int64_t(1) << 31) - 1 || Lk > (int64_t(1) << 31) - 1)
+    return HSA_ERR_ARG;
+  if (Lq == 0) return HSA_OK;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(indices) || !aligned16(O))
+    return HSA_ERR_ARG;
+  if (int e = check_device()) return e;
+  hsa::RowMap rm{Lq, Lk, nullptr, 0};
+  hsa::launch_sparse_attn_simple(rm, Lq, Q, K, V, indices, p->k, p->H, p->d, softmax_scale(p), O,
+                                 stream);
+  return launch_status();
+}
+
+int hsa_decode_workspace_size(const hsa_params* p, int32_t batch, int64_t capacity,
+                              size_t* bytes) {
+  if (!bytes) return HSA_ERR_ARG;
+  if (int e = check_index_params(p)) return e;
+  if (int e = check_attn_params(p)) return e;
+  if (batch < 0 || capacity < p->B || capacity % p->B) return HSA_ERR_ARG;
+  *bytes = align_up(size_t(batch) * p->m * sizeof(int32_t)) +
+           align_up(size_t(batch) * p->k * sizeof(int32_t));
+  return HSA_OK;
+}
+
+int hsa_decode_step(const hsa_params* p, int32_t batch, int64_t capacity, int32_t* ctx_len,
+                    hsa_bf16* k_idx_cache, hsa_bf16* K_cache, hsa_bf16* V_cache,
+                    float* ksum_cache, const hsa_bf16* q_idx_new, const hsa_bf16* k_idx_new,
+                    const hsa_bf16* Q_new, const hsa_bf16* K_new, const hsa_bf16* V_new,
+                    hsa_bf16* O, int32_t* indices_out, void* workspace, size_t workspace_bytes,
+                    cudaStream_t stream) {
+  size_t need = 0;
+  if (int e = hsa_decode_workspace_size(p, batch, capacity, &need)) return e;
+  if (capacity / p->B > kMaxCandidates || capacity > (int64_t(1) << 31) - 1) return HSA_ERR_ARG;
+  if (batch == 0) return HSA_OK;
+  const void* ptrs[] = {ctx_len, k_idx_cache, K_cache, V_cache, ksum_cache, q_idx_new,
+                        k_idx_new, Q_new, K_new, V_new, O};
+  for (const void* q : ptrs)
+    if (!aligned16(q) && q != ctx_len) return HSA_ERR_ARG;
+  if (!ctx_len || (reinterpret_cast<uintptr_t>(ctx_len) & 3u)) return HSA_ERR_ARG;
+  if (indices_out && !aligned16(indices_out)) return HSA_ERR_ARG;
+  if (!aligned16(workspace) || workspace_bytes < need) return HSA_ERR_WORKSPACE;
+  if (int e = check_device()) return e;
+  char* ws = static_cast<char*>(workspace);
+  int32_t* blocks = reinterpret_cast<int32_t*>(ws);
+  int32_t* idx = indices_out ? indices_out
+                             : reinterpret_cast<int32_t*>(ws + align_up(size_t(batch) * p->m * 4));
+  hsa::launch_decode_append(batch, capacity, ctx_len, p->B, p->d_idx, p->d, k_idx_cache, K_cache,
+                            V_cache, ksum_cache, k_idx_new, K_new, V_new, stream);
+  hsa::RowMap rm{batch, capacity, ctx_len, capacity};
+  hsa::launch_select_blocks(rm, batch, q_idx_new, ksum_cache, (capacity / p->B) * p->d_idx, p->B,
+                            p->m, p->d_idx, blocks, capacity / p->B, stream);
+  hsa::launch_select_tokens(rm, batch, q_idx_new, k_idx_cache, blocks, p->B, p->m, p->k,
+                            p->d_idx, idx, stream);
+  hsa::launch_sparse_attn_simple(rm, batch, Q_new, K_cache, V_cache, idx, p->k, p->H, p->d,
+                                 softmax_scale(p), O, stream);
+  hsa::launch_decode_advance(batch, capacity, ctx_len, stream);
+  return launch_status();
+}
+
+}  // extern "C"

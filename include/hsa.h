@@ -1,0 +1,169 @@
+/*
+ * hsa.h -- C ABI of the B200 (sm_100a) hierarchical indexed sparse attention
+ * (HISA) library, libhsa.so.
+ *
+ * The method (page "HISA: Hierarchical Indexed Sparse Attention",
+ * discuz.ruhao.net thread 187): a drop-in replacement for the token-level
+ * indexer of DeepSeek sparse attention (DSA). For every query position t the
+ * causal key prefix is cut into blocks of B tokens (section 第一步); each block
+ * gets a representative vector, the blocks are scored with the indexer's own
+ * rule and the best m are kept, the first block and the query's own (last)
+ * block always among them (the forced first/last block note). Only the
+ * tokens inside the kept blocks are then scored and the best k kept
+ * (section 第二步); the output has the original indexer's format and the
+ * attention that follows is the unchanged sparse softmax attention over those
+ * k tokens, shared by all H query heads of a multi-query layer (the
+ * "drop-in replacement" paragraph). The indexer cost falls from O(L^2) to
+ * O(L^2/B + L*m*B) (the complexity paragraph).
+ *
+ * Readings fixed by this library where the pages are silent:
+ *   - scoring rule: plain dot product q_idx[t] . k_idx[j] (one indexer head);
+ *   - block representative: fp32 sum of the block's B key rows;
+ *   - the m kept blocks include the two forced ones; the other m-2 are the
+ *     best-scoring complete blocks among 1 .. floor(t/B)-1;
+ *   - causal keys are j <= t; ties go to the lowest index;
+ *   - indices are written ascending and padded with -1;
+ *   - softmax scale defaults to 1/sqrt(d).
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers to dense row-major arrays owned
+ *     by the caller; the library never allocates, frees or synchronises on the
+ *     hot path. bf16 tensors are passed as 16-bit bit patterns (hsa_bf16).
+ *   - Pointers must be 16-byte aligned and the row lengths below must keep
+ *     every row 16-byte aligned (d_idx and d are multiples of 8).
+ *   - Work is enqueued on `stream`; the call returns once it is enqueued.
+ *   - Every argument is checked on the host before anything is launched; on
+ *     a failed check nothing is launched and an HSA_ERR_* code is returned.
+ *     No exception crosses this boundary. Non-finite inputs are not checked.
+ *   - Indexer inputs holding integer values of magnitude <= 8 (the synthetic
+ *     workloads) give exact fp32 scores, so selections are reproducible bit
+ *     for bit; for general real inputs near-ties may order differently from a
+ *     sequential CPU evaluation.
+ */
+#ifndef HSA_H_
+#define HSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define HSA_API __attribute__((visibility("default")))
+#else
+#define HSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t hsa_bf16; /* bf16 bit pattern */
+
+enum {
+  HSA_OK = 0,
+  HSA_ERR_ARG = 1,       /* null / misaligned pointer or unsupported size  */
+  HSA_ERR_WORKSPACE = 2, /* workspace missing or smaller than required      */
+  HSA_ERR_CUDA = 3,      /* a CUDA launch or runtime call failed            */
+  HSA_ERR_TIMEOUT = 4,   /* a bounded device-side wait gave up              */
+  HSA_ERR_DEVICE = 5     /* current device is not sm_100 (B200 class)       */
+};
+
+/* Method and layer sizes. */
+typedef struct hsa_params {
+  int32_t B;     /* tokens per block, 1 <= B <= 1024                           */
+  int32_t m;     /* kept blocks per query incl. the 2 forced ones, 2 <= m <= 256 */
+  int32_t k;     /* kept tokens per query, 1 <= k <= 8192, k <= m*B            */
+  int32_t d_idx; /* indexer head dim: 64 or 128                                 */
+  int32_t H;     /* query heads sharing one K/V head: 1 <= H <= 128             */
+  int32_t d;     /* attention head dim: 64 or 128                               */
+  float scale;   /* softmax scale; 0 selects 1/sqrt(d)                          */
+} hsa_params;
+
+/* Human-readable text for a status code (static storage). */
+HSA_API const char* hsa_status_string(int status);
+
+/* Workspace bytes needed by hsa_index / hsa_select_blocks / hsa_select_tokens
+ * for Lq queries over Lk keys. Writes *bytes. */
+HSA_API int hsa_index_workspace_size(const hsa_params* p, int64_t Lq, int64_t Lk, size_t* bytes);
+
+/* Block representatives (section 第一步).
+ *   k_idx [Lk][d_idx] bf16 keys of the indexer.
+ *   ksum  [floor(Lk/B)][d_idx] fp32, written: ksum[b][c] = sum_{j in block b} k_idx[j][c].
+ * Only complete blocks are produced. */
+HSA_API int hsa_block_sums(const hsa_params* p, int64_t Lk, const hsa_bf16* k_idx, float* ksum,
+                   cudaStream_t stream);
+
+/* Block-level selection (section 第一步 + forced first/last block).
+ * Query i (0 <= i < Lq) sits at absolute position t = Lk - Lq + i.
+ *   q_idx  [Lq][d_idx] bf16 indexer queries.
+ *   ksum   [floor(Lk/B)][d_idx] fp32 from hsa_block_sums.
+ *   blocks [Lq][m] int32, written: kept block ids ascending, -1 padded.
+ * With nb = floor(t/B)+1 causal blocks: nb <= m keeps them all; otherwise
+ * blocks 0 and nb-1 plus the m-2 best of 1..nb-2 by (score desc, id asc). */
+HSA_API int hsa_select_blocks(const hsa_params* p, int64_t Lq, int64_t Lk, const hsa_bf16* q_idx,
+                      const float* ksum, int32_t* blocks, void* workspace,
+                      size_t workspace_bytes, cudaStream_t stream);
+
+/* Token-level selection inside the kept blocks (section 第二步).
+ *   q_idx [Lq][d_idx], k_idx [Lk][d_idx] bf16; blocks [Lq][m] from hsa_select_blocks.
+ *   indices [Lq][k] int32, written ascending, -1 padded.
+ * Candidates are the tokens j <= t of the kept blocks; if there are at most k
+ * of them all are kept, else the k best by (score desc, j asc). */
+HSA_API int hsa_select_tokens(const hsa_params* p, int64_t Lq, int64_t Lk, const hsa_bf16* q_idx,
+                      const hsa_bf16* k_idx, const int32_t* blocks, int32_t* indices,
+                      void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* The whole indexer: block sums, block selection and token selection.
+ *   q_idx [Lq][d_idx], k_idx [Lk][d_idx] bf16 -> indices [Lq][k] int32.
+ * Requires 1 <= Lq <= Lk. workspace: hsa_index_workspace_size bytes. */
+HSA_API int hsa_index(const hsa_params* p, int64_t Lq, int64_t Lk, const hsa_bf16* q_idx,
+              const hsa_bf16* k_idx, int32_t* indices, void* workspace, size_t workspace_bytes,
+              cudaStream_t stream);
+
+/* Sparse softmax attention over the kept tokens (the unchanged downstream
+ * attention of the "drop-in replacement" paragraph; softmax(q K^T * scale) V
+ * as in the HiLS page's Step 4), multi-query: all H heads share the indices.
+ *   Q [Lq][H][d] bf16; K, V [Lk][d] bf16; indices [Lq][k] int32 (entries < 0
+ *   are skipped, entries must be < Lk); O [Lq][H][d] bf16, written.
+ * fp32 accumulation, O rounded once to bf16. A row without any valid index
+ * yields zeros. */
+HSA_API int hsa_sparse_attn(const hsa_params* p, int64_t Lq, int64_t Lk, const hsa_bf16* Q,
+                    const hsa_bf16* K, const hsa_bf16* V, const int32_t* indices, hsa_bf16* O,
+                    cudaStream_t stream);
+
+/* Workspace bytes for hsa_decode_step. */
+HSA_API int hsa_decode_workspace_size(const hsa_params* p, int32_t batch, int64_t capacity,
+                              size_t* bytes);
+
+/* One decode step for `batch` independent sequences (the decode regime the
+ * pages describe as one query per step over a growing KV cache).
+ * Caches (device, caller-owned, `capacity` rows per sequence, capacity a
+ * multiple of B):
+ *   k_idx_cache [batch][capacity][d_idx] bf16, K_cache/V_cache [batch][capacity][d] bf16,
+ *   ksum_cache  [batch][capacity/B][d_idx] fp32 (block sums of complete blocks;
+ *               fill it for the prompt with hsa_block_sums),
+ *   ctx_len     [batch] int32: cached tokens per sequence.
+ * New token per sequence: q_idx_new/k_idx_new [batch][d_idx], Q_new [batch][H][d],
+ *   K_new/V_new [batch][d] (all bf16).
+ * The step appends the new token at position t = ctx_len[b], writes the
+ * block sum of a block the token completes, selects blocks and tokens for
+ * the query at t (keys j <= t), attends, writes O [batch][H][d] bf16 and,
+ * if indices_out is not NULL, the kept indices [batch][k]; then ctx_len[b]
+ * += 1. A sequence with ctx_len[b] >= capacity is left untouched and its O
+ * row is zero. */
+HSA_API int hsa_decode_step(const hsa_params* p, int32_t batch, int64_t capacity, int32_t* ctx_len,
+                    hsa_bf16* k_idx_cache, hsa_bf16* K_cache, hsa_bf16* V_cache,
+                    float* ksum_cache, const hsa_bf16* q_idx_new, const hsa_bf16* k_idx_new,
+                    const hsa_bf16* Q_new, const hsa_bf16* K_new, const hsa_bf16* V_new,
+                    hsa_bf16* O, int32_t* indices_out, void* workspace, size_t workspace_bytes,
+                    cudaStream_t stream);
+
+/* Number of kernels this library has launched in the calling process (all
+ * devices, all streams) since it was loaded. A diagnostic counter for
+ * benchmarks and tests; it is not synchronised with the GPU. */
+HSA_API uint64_t hsa_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HSA_H_ */

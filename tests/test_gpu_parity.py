@@ -1,0 +1,273 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Selected indices and block lists must match bit for bit (integer-valued
+indexer inputs make every fp32 score exact); attention outputs must be within
+max-abs 2e-2 / mean-abs 2e-3 of the oracle's fp64 result.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from helpers import assert_attn_close, dev, host_bits, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def hsa():
+    import torch
+    import hierarchical_sparse_attention_hisa_b200 as m
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    m.build()
+    m.load()
+    return m
+
+
+def run_index(hsa, q, k, B, m, kk):
+    import torch
+    out = hsa.index(dev(q), dev(k), B, m, kk)
+    torch.cuda.synchronize()
+    return out.cpu().numpy()
+
+
+def run_attn(hsa, Q, K, V, idx_np, scale=0.0):
+    import torch
+    idx = torch.from_numpy(np.ascontiguousarray(idx_np, dtype=np.int32)).cuda()
+    O = hsa.sparse_attn(dev(Q), dev(K), dev(V), idx, scale=scale)
+    torch.cuda.synchronize()
+    return host_bits(O)
+
+
+# ------------------------------------------------------------------ stages
+
+@pytest.mark.parametrize("Lk,B,d", [(2048, 64, 64), (5037, 128, 128), (999, 7, 64), (64, 64, 128)])
+def test_block_sums_bit_exact(hsa, Lk, B, d):
+    import torch
+    k = synth.int_bf16((Lk, d), 11, 2)
+    ks = torch.empty((Lk // B, d), dtype=torch.float32, device="cuda")
+    p = hsa.params(B=B, m=8, k=16, d_idx=d)
+    hsa.hsa_block_sums(p, Lk, dev(k), ks)
+    torch.cuda.synchronize()
+    assert np.array_equal(ks.cpu().numpy(), oracle.block_sums(k, B))
+
+
+@pytest.mark.parametrize("Lq,Lk,B,m,d", [(2048, 2048, 64, 8, 64), (700, 5037, 128, 6, 128),
+                                         (300, 300, 4, 2, 64), (4096, 4096, 16, 40, 128)])
+def test_select_blocks_bit_exact(hsa, Lq, Lk, B, m, d):
+    import torch
+    q, k = synth.int_bf16((Lq, d), 12, 1), synth.int_bf16((Lk, d), 12, 2)
+    p = hsa.params(B=B, m=m, k=16, d_idx=d)
+    ks = torch.empty((max(Lk // B, 1), d), dtype=torch.float32, device="cuda")
+    hsa.hsa_block_sums(p, Lk, dev(k), ks)
+    blocks = torch.empty((Lq, m), dtype=torch.int32, device="cuda")
+    hsa.hsa_select_blocks(p, Lq, Lk, dev(q), ks, blocks)
+    torch.cuda.synchronize()
+    want = oracle.select_blocks(q, oracle.block_sums(k, B), Lk, B, m)
+    assert np.array_equal(blocks.cpu().numpy(), want)
+
+
+# ------------------------------------------------------------------ indexer
+
+def test_index_tiny_prefill_all_rows(hsa):
+    w = synth.WORKLOADS["tiny_prefill_2k"]
+    x = synth.prefill_inputs(w, with_attn=False)
+    got = run_index(hsa, x["q_idx"], x["k_idx"], w.B, w.m, w.k)
+    assert np.array_equal(got, oracle.index(x["q_idx"], x["k_idx"], w.B, w.m, w.k))
+
+
+def test_index_prefill_16k_all_rows(hsa):
+    w = synth.WORKLOADS["prefill_16k"]
+    x = synth.prefill_inputs(w, with_attn=False)
+    got = run_index(hsa, x["q_idx"], x["k_idx"], w.B, w.m, w.k)
+    want = oracle.index(x["q_idx"], x["k_idx"], w.B, w.m, w.k)
+    bad = np.nonzero((got != want).any(axis=1))[0]
+    assert len(bad) == 0, f"{len(bad)} rows differ, first {bad[:5]}"
+
+
+@pytest.mark.parametrize("Lq,Lk,B,m,k,d", [
+    (777, 5037, 64, 8, 256, 128),     # chunk of queries, ragged last block
+    (1, 1, 64, 8, 256, 64),           # a single token
+    (1, 9000, 128, 16, 2048, 128),    # one query at the end of a long prefix
+    (512, 512, 16, 2, 7, 64),         # m = 2: forced blocks only
+    (600, 600, 32, 4, 1, 64),         # k = 1
+    (400, 400, 8, 5, 40, 128),        # k = m*B: every candidate of a full row kept
+    (333, 1000, 10, 12, 100, 64),     # B not a power of two
+])
+def test_index_shapes_bit_exact(hsa, Lq, Lk, B, m, k, d):
+    q, kk = synth.int_bf16((Lq, d), 13, 1), synth.int_bf16((Lk, d), 13, 2)
+    got = run_index(hsa, q, kk, B, m, k)
+    assert np.array_equal(got, oracle.index(q, kk, B, m, k))
+
+
+def test_index_all_ties_goes_to_lowest_indices(hsa):
+    Lq = Lk = 1500
+    q = np.zeros((Lq, 64), dtype=np.uint16)     # every score is 0
+    kk = synth.int_bf16((Lk, 64), 14, 2)
+    got = run_index(hsa, q, kk, 32, 6, 50)
+    assert np.array_equal(got, oracle.index(q, kk, 32, 6, 50))
+
+
+def test_index_extreme_magnitudes_exact(hsa):
+    # all entries +-8: token scores reach +-8192 and block scores +-2^20
+    rng = np.random.default_rng(15)
+    Lq = Lk = 4096
+    q = synth.f32_to_bf16_bits(rng.choice([-8.0, 8.0], size=(Lq, 128)).astype(np.float32))
+    kk = synth.f32_to_bf16_bits(rng.choice([-8.0, 8.0], size=(Lk, 128)).astype(np.float32))
+    kk[:128] = synth.f32_to_bf16_bits(np.full((128, 128), 8.0, np.float32))
+    q[-1] = synth.f32_to_bf16_bits(np.full(128, 8.0, np.float32))
+    got = run_index(hsa, q, kk, 128, 8, 512)
+    assert np.array_equal(got, oracle.index(q, kk, 128, 8, 512))
+
+
+def test_index_prefill_64k_sampled_rows_and_needles(hsa):
+    w = synth.WORKLOADS["prefill_64k"]
+    x = synth.prefill_inputs(w, with_attn=False)
+    got = run_index(hsa, x["q_idx"], x["k_idx"], w.B, w.m, w.k)
+    needle_rows = [i for i, _ in x["needles"]]
+    rows = sample_rows(w.Lq, 384, 16, always=[0, 1, 2047, 2048, 8191, 8192, w.Lq - 1, *needle_rows])
+    want = oracle.index(x["q_idx"], x["k_idx"], w.B, w.m, w.k, rows=rows)
+    assert np.array_equal(got[rows], want)
+    # structural checks on every row: ascending, causal, -1 only as tail padding
+    t = np.arange(w.Lq)[:, None]
+    valid = got >= 0
+    assert (got <= t).all()
+    assert (np.diff(np.where(valid, got, np.iinfo(np.int32).max), axis=1) > 0).all()
+    recall = np.mean([j in set(got[i].tolist()) for i, j in x["needles"]])
+    print(f"needle recall {recall:.3f}")
+
+
+def test_index_long_context_chunk_sampled(hsa):
+    w = synth.WORKLOADS["prefill_1m_last8k"]
+    x = synth.prefill_inputs(w, with_attn=False)
+    got = run_index(hsa, x["q_idx"], x["k_idx"], w.B, w.m, w.k)
+    rows = sample_rows(w.Lq, 96, 17, always=[0, w.Lq - 1])
+    want = oracle.index(x["q_idx"], x["k_idx"], w.B, w.m, w.k, rows=rows)
+    assert np.array_equal(got[rows], want)
+
+
+# ------------------------------------------------------------------ attention
+
+def test_attention_tiny_prefill_all_rows(hsa):
+    w = synth.WORKLOADS["tiny_prefill_2k"]
+    x = synth.prefill_inputs(w)
+    idx = oracle.index(x["q_idx"], x["k_idx"], w.B, w.m, w.k)
+    got = run_attn(hsa, x["Q"], x["K"], x["V"], idx)
+    ref = oracle.sparse_attn(x["Q"], x["K"], x["V"], idx)
+    print("tiny max/mean abs err", assert_attn_close(got, ref, "tiny"))
+
+
+def test_attention_prefill_16k_sampled(hsa):
+    w = synth.WORKLOADS["prefill_16k"]
+    x = synth.prefill_inputs(w)
+    idx = run_index(hsa, x["q_idx"], x["k_idx"], w.B, w.m, w.k)
+    got = run_attn(hsa, x["Q"], x["K"], x["V"], idx)
+    rows = sample_rows(w.Lq, 512, 18, always=[0, 1, 100, 2047, 2048, w.Lq - 1])
+    ref = oracle.sparse_attn(x["Q"], x["K"], x["V"], idx[rows], rows=rows)
+    print("16k max/mean abs err", assert_attn_close(got[rows], ref, "16k"))
+
+
+@pytest.mark.parametrize("H,d,k", [(1, 64, 5), (16, 128, 1), (64, 128, 300), (128, 64, 130),
+                                   (8, 128, 2048)])
+def test_attention_shapes(hsa, H, d, k):
+    Lq, Lk = 70, 3000
+    rng = np.random.default_rng(H * 1000 + k)
+    Q, K, V = (synth.normal_bf16(s, 19, i) for i, s in enumerate([(Lq, H, d), (Lk, d), (Lk, d)]))
+    idx = np.full((Lq, k), -1, dtype=np.int32)
+    for i in range(Lq):
+        n = int(rng.integers(0, k + 1)) if i % 7 else k   # ragged rows, some empty
+        idx[i, :n] = np.sort(rng.choice(Lk, size=n, replace=False))
+    got = run_attn(hsa, Q, K, V, idx)
+    ref = oracle.sparse_attn(Q, K, V, idx)
+    assert_attn_close(got, ref, f"H={H} d={d} k={k}")
+
+
+def test_attention_large_logits_stable(hsa):
+    # Q, K of magnitude 4..8: scaled logits in the hundreds; exact softmax must hold.
+    Lq, Lk, H, d, k = 16, 512, 4, 128, 256
+    rng = np.random.default_rng(20)
+    Q = synth.f32_to_bf16_bits((rng.choice([-1, 1], size=(Lq, H, d)) * 6.0).astype(np.float32))
+    K = synth.f32_to_bf16_bits((rng.choice([-1, 1], size=(Lk, d)) * 4.0).astype(np.float32))
+    V = synth.normal_bf16((Lk, d), 20, 5)
+    idx = np.stack([np.sort(rng.choice(Lk, size=k, replace=False)) for _ in range(Lq)]).astype(np.int32)
+    got = run_attn(hsa, Q, K, V, idx)
+    assert_attn_close(got, oracle.sparse_attn(Q, K, V, idx), "large logits")
+
+
+def test_attention_explicit_scale(hsa):
+    Lq, Lk, H, d, k = 20, 400, 4, 64, 64
+    Q, K, V = (synth.normal_bf16(s, 21, i) for i, s in enumerate([(Lq, H, d), (Lk, d), (Lk, d)]))
+    rng = np.random.default_rng(21)
+    idx = np.stack([np.sort(rng.choice(Lk, size=k, replace=False)) for _ in range(Lq)]).astype(np.int32)
+    got = run_attn(hsa, Q, K, V, idx, scale=0.3)
+    assert_attn_close(got, oracle.sparse_attn(Q, K, V, idx, scale=0.3), "scale")
+
+
+def test_attention_prefill_64k_sampled(hsa):
+    w = synth.WORKLOADS["prefill_64k"]
+    x = synth.prefill_inputs(w)
+    idx = run_index(hsa, x["q_idx"], x["k_idx"], w.B, w.m, w.k)
+    got = run_attn(hsa, x["Q"], x["K"], x["V"], idx)
+    rows = sample_rows(w.Lq, 192, 22, always=[0, 1, 2047, w.Lq - 1])
+    ref = oracle.sparse_attn(x["Q"], x["K"], x["V"], idx[rows], rows=rows)
+    print("64k max/mean abs err", assert_attn_close(got[rows], ref, "64k"))
+
+
+# ------------------------------------------------------------------ decode
+
+def decode_case(hsa, B, m, k, d_idx, H, d, ctx0, capacity, steps, seed, check_seqs=None):
+    """Run `steps` decode steps on the GPU and compare every step with the
+    oracle evaluated on the host copy of each sequence's cache."""
+    import torch
+    batch = len(ctx0)
+    rng = np.random.default_rng(seed)
+    kc = synth.int_bf16((batch, capacity, d_idx), seed, 2)
+    Kc = synth.normal_bf16((batch, capacity, d), seed, 4)
+    Vc = synth.normal_bf16((batch, capacity, d), seed, 5)
+    new = {n: synth.int_bf16((steps, batch, d_idx), seed, 30 + i) for i, n in enumerate(["q", "k"])}
+    newQ = synth.normal_bf16((steps, batch, H, d), seed, 33)
+    newK = synth.normal_bf16((steps, batch, d), seed, 34)
+    newV = synth.normal_bf16((steps, batch, d), seed, 35)
+    p = hsa.params(B=B, m=m, k=k, d_idx=d_idx, H=H, d=d)
+    g_kc, g_Kc, g_Vc = dev(kc), dev(Kc), dev(Vc)
+    ksum = torch.zeros((batch, capacity // B, d_idx), dtype=torch.float32, device="cuda")
+    for b in range(batch):
+        hsa.hsa_block_sums(p, int(ctx0[b]), g_kc[b], ksum[b])
+    ctx = torch.tensor(ctx0, dtype=torch.int32, device="cuda")
+    ws = torch.empty(hsa.hsa_decode_workspace_size(p, batch, capacity), dtype=torch.uint8, device="cuda")
+    O = torch.empty((batch, H, d), dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty((batch, k), dtype=torch.int32, device="cuda")
+    lens = np.array(ctx0, dtype=np.int64)
+    check = range(batch) if check_seqs is None else check_seqs
+    for s in range(steps):
+        hsa.hsa_decode_step(p, batch, capacity, ctx, g_kc, g_Kc, g_Vc, ksum, dev(new["q"][s]),
+                            dev(new["k"][s]), dev(newQ[s]), dev(newK[s]), dev(newV[s]), O, idx, ws)
+        torch.cuda.synchronize()
+        got_idx, got_O = idx.cpu().numpy(), host_bits(O)
+        for b in check:
+            t = int(lens[b])
+            if t >= capacity:
+                assert (got_idx[b] == -1).all() and (got_O[b] == 0).all()
+                continue
+            kc[b, t], Kc[b, t], Vc[b, t] = new["k"][s, b], newK[s, b], newV[s, b]
+            want = oracle.index(new["q"][s, b][None], kc[b, : t + 1], B, m, k)
+            assert np.array_equal(got_idx[b], want[0]), (s, b)
+            ref = oracle.sparse_attn(newQ[s, b][None], Kc[b, : t + 1], Vc[b, : t + 1], want)
+            assert_attn_close(got_O[b][None], ref, f"decode step {s} seq {b}")
+        lens = np.minimum(lens + 1, capacity)
+        assert np.array_equal(ctx.cpu().numpy(), np.minimum(np.array(ctx0) + s + 1, capacity))
+    # block sums written by the steps match the oracle's for every complete block
+    for b in check:
+        n = int(lens[b]) // B
+        assert np.array_equal(ksum[b, :n].cpu().numpy(), oracle.block_sums(kc[b, : n * B], B))
+
+
+def test_decode_small_all_sequences(hsa):
+    # ragged lengths, block completions during the run, one sequence hitting capacity
+    decode_case(hsa, B=64, m=8, k=256, d_idx=64, H=4, d=64, ctx0=[1, 63, 500, 1000, 1020],
+                capacity=1024, steps=70, seed=40)
+
+
+def test_decode_128k_two_steps_sampled(hsa):
+    decode_case(hsa, B=128, m=64, k=2048, d_idx=128, H=64, d=128, ctx0=[131072] * 32,
+                capacity=131072 + 256, steps=2, seed=41, check_seqs=[0, 7, 31])
