@@ -191,9 +191,14 @@ int hsa_sparse_attn(const hsa_params* p, int64_t Lq, int64_t Lk, const hsa_bf16*
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(indices) || !aligned16(O))
     return HSA_ERR_ARG;
   if (int e = check_device()) return e;
-  hsa::RowMap rm{Lq, Lk, nullptr, 0};
-  hsa::launch_sparse_attn_simple(rm, Lq, Q, K, V, indices, p->k, p->H, p->d, softmax_scale(p), O,
-                                 stream);
+  if (hsa::tc_attn_supported(p->H, p->d, Lq, Lk)) {
+    if (!hsa::launch_sparse_attn_tc(Lq, Q, K, V, indices, Lk, p->k, p->H, softmax_scale(p), O, stream))
+      return HSA_ERR_CUDA;
+  } else {
+    hsa::RowMap rm{Lq, Lk, nullptr, 0};
+    hsa::launch_sparse_attn_simple(rm, Lq, Q, K, V, indices, p->k, p->H, p->d, softmax_scale(p), O,
+                                   stream);
+  }
   return launch_status();
 }
 

@@ -77,6 +77,10 @@ __global__ void __launch_bounds__(256) select_blocks_kernel(RowMap rm, const uin
     for (int s = threadIdx.x; s < m; s += NT) out[s] = s < nb ? s : -1;
     return;
   }
+  if (m == 2) {  // only the two forced blocks are kept
+    if (threadIdx.x == 0) { out[0] = 0; out[1] = int32_t(nb - 1); }
+    return;
+  }
   for (int c = threadIdx.x; c < D; c += NT) qs[c] = __uint_as_float(uint32_t(q_idx[i * D + c]) << 16);
   __syncthreads();
   const float* ks = ksum + (rm.ctx ? i * ksum_seq_stride : 0);

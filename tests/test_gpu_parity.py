@@ -132,7 +132,11 @@ def test_index_prefill_64k_sampled_rows_and_needles(hsa):
     t = np.arange(w.Lq)[:, None]
     valid = got >= 0
     assert (got <= t).all()
-    assert (np.diff(np.where(valid, got, np.iinfo(np.int32).max), axis=1) > 0).all()
+    nvalid = valid.sum(axis=1)
+    assert (valid == (np.arange(w.k)[None, :] < nvalid[:, None])).all()  # -1 only as a tail
+    assert (nvalid == np.minimum(np.arange(w.Lq) + 1, w.k)).all()
+    inc = np.diff(got, axis=1) > 0
+    assert (inc | ~valid[:, 1:]).all()  # strictly ascending over the valid prefix
     recall = np.mean([j in set(got[i].tolist()) for i, j in x["needles"]])
     print(f"needle recall {recall:.3f}")
 
@@ -201,6 +205,47 @@ def test_attention_explicit_scale(hsa):
     idx = np.stack([np.sort(rng.choice(Lk, size=k, replace=False)) for _ in range(Lq)]).astype(np.int32)
     got = run_attn(hsa, Q, K, V, idx, scale=0.3)
     assert_attn_close(got, oracle.sparse_attn(Q, K, V, idx, scale=0.3), "scale")
+
+
+def test_attention_explicit_scale_d128(hsa):
+    Lq, Lk, H, d, k = 33, 900, 64, 128, 257
+    Q, K, V = (synth.normal_bf16(s, 23, i) for i, s in enumerate([(Lq, H, d), (Lk, d), (Lk, d)]))
+    rng = np.random.default_rng(23)
+    idx = np.stack([np.sort(rng.choice(Lk, size=k, replace=False)) for _ in range(Lq)]).astype(np.int32)
+    got = run_attn(hsa, Q, K, V, idx, scale=0.05)
+    assert_attn_close(got, oracle.sparse_attn(Q, K, V, idx, scale=0.05), "scale d128")
+
+
+def test_attention_holes_and_out_of_range_entries(hsa):
+    # -1 entries anywhere in a row (not only as a tail) are skipped
+    Lq, Lk, H, d, k = 40, 2000, 16, 128, 700
+    Q, K, V = (synth.normal_bf16(s, 24, i) for i, s in enumerate([(Lq, H, d), (Lk, d), (Lk, d)]))
+    rng = np.random.default_rng(24)
+    idx = np.stack([np.sort(rng.choice(Lk, size=k, replace=False)) for _ in range(Lq)]).astype(np.int32)
+    idx[rng.random(idx.shape) < 0.3] = -1
+    idx[5, :] = -1            # an empty row
+    idx[6, 130:] = -1         # only the first tile valid
+    idx[7, :600] = -1         # only the last tiles valid
+    got = run_attn(hsa, Q, K, V, idx)
+    ref = oracle.sparse_attn(Q, K, V, idx)
+    assert (got[5] == 0).all()
+    assert_attn_close(got, ref, "holes")
+
+
+@pytest.mark.parametrize("H", [64, 16, 5])
+def test_attention_running_max_rescales(hsa, H):
+    # scores grow by ~8 (log2 units) from one 128-key tile to the next, so the
+    # running maximum is raised and the accumulator rescaled on every tile
+    Lq, Lk, d, k = 12, 2048, 128, 2048
+    Q = synth.f32_to_bf16_bits(np.ones((Lq, H, d), np.float32)
+                               * (1.0 + np.arange(H, dtype=np.float32) / 64)[None, :, None])
+    K = synth.f32_to_bf16_bits(np.repeat(0.5 * (np.arange(Lk) // 128), d).reshape(Lk, d).astype(np.float32))
+    V = synth.normal_bf16((Lk, d), 25, 5)
+    idx = np.tile(np.arange(k, dtype=np.int32), (Lq, 1))
+    idx[1, 1000:] = -1
+    idx[2] = idx[2][::-1].copy()  # descending order: the first tile holds the maximum
+    got = run_attn(hsa, Q, K, V, idx)
+    assert_attn_close(got, oracle.sparse_attn(Q, K, V, idx), "rescale")
 
 
 def test_attention_prefill_64k_sampled(hsa):
