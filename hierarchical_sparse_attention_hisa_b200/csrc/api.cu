@@ -71,22 +71,103 @@ int launch_status() {
   return cudaGetLastError() == cudaSuccess ? HSA_OK : HSA_ERR_CUDA;
 }
 
-struct IndexWs {
-  size_t ksum_off, blocks_off, total;
-};
-IndexWs index_ws(const hsa_params* p, int64_t Lq, int64_t Lk) {
-  IndexWs w;
-  w.ksum_off = 0;
-  w.blocks_off = align_up(size_t(Lk / p->B) * p->d_idx * sizeof(float));
-  w.total = w.blocks_off + align_up(size_t(Lq) * p->m * sizeof(int32_t));
-  return w;
-}
-
 // Largest number of block candidates any query of [Lk-Lq, Lk) scores.
 int64_t max_block_candidates(const hsa_params* p, int64_t Lk) {
   const int64_t nb = (Lk - 1) / p->B + 1;
   return nb > 2 ? nb - 2 : 1;
 }
+
+// Workspace of the indexer (all offsets 256-byte aligned):
+//   ksum   [nbc][d_idx] fp32          block sums
+//   bsplit [3][nbc][d_idx] bf16       hi/mid/lo planes of ksum
+//   bkeys  [Lq][ldb] u32              block-score keys (ldb = nbc rounded to 64)
+//   blocks [Lq][m] i32                kept blocks
+//   cnt/off/cursor [nbins] i32        pairs per key block (nbins = ceil(Lk/B))
+//   ntiles i32, tiles [max_tiles] int4, pairs [Lq*m] u32
+//   tkeys  [Lq][m][B] u32             token-score keys
+struct IndexWs {
+  size_t ksum, bsplit, bkeys, blocks, cnt, off, cursor, ntiles, tiles, pairs, tkeys, total;
+  int64_t nbc, ldb, nbins, max_tiles;
+};
+IndexWs index_ws(const hsa_params* p, int64_t Lq, int64_t Lk) {
+  IndexWs w{};
+  w.nbc = Lk / p->B;
+  w.ldb = (w.nbc + 63) / 64 * 64;
+  w.nbins = (Lk + p->B - 1) / p->B;
+  w.max_tiles = (Lq * p->m + 127) / 128 + w.nbins;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { const size_t at = o; o += align_up(bytes > 0 ? bytes : 1); return at; };
+  w.ksum = take(size_t(w.nbc) * p->d_idx * 4);
+  w.bsplit = take(size_t(3) * w.nbc * p->d_idx * 2);
+  w.bkeys = take(size_t(Lq) * w.ldb * 4);
+  w.blocks = take(size_t(Lq) * p->m * 4);
+  w.cnt = take(size_t(w.nbins) * 4);
+  w.off = take(size_t(w.nbins) * 4);
+  w.cursor = take(size_t(w.nbins) * 4);
+  w.ntiles = take(16);
+  w.tiles = take(size_t(w.max_tiles) * 16);
+  w.pairs = take(size_t(Lq) * p->m * 4);
+  w.tkeys = take(size_t(Lq) * p->m * p->B * 4);
+  w.total = o;
+  return w;
+}
+
+// Tensor-core scoring covers d_idx in {64, 128}; block scoring needs a full
+// 128-query tile and at least 64 rows of split block sums, token scoring a
+// block size the MMA N dimension can take and one full key block.
+bool block_gemm_ok(const hsa_params* p, int64_t Lq, int64_t Lk) {
+  return Lq >= 128 && 3 * (Lk / p->B) >= 64;
+}
+bool token_gemm_ok(const hsa_params* p, int64_t Lq, int64_t Lk) {
+  return (p->B == 64 || p->B == 128) && Lk >= p->B && Lq * int64_t(p->m) < (int64_t(1) << 32);
+}
+
+// Kept blocks for rows [0, Lq) from fp32 block sums.
+void run_select_blocks(const hsa_params* p, int64_t Lq, int64_t Lk, const void* q_idx, const float* ksum,
+                       int32_t* blocks, char* ws, const IndexWs& w, cudaStream_t s, bool* ok) {
+  hsa::RowMap rm{Lq, Lk, nullptr, 0};
+  const int64_t nb_last = (Lk - 1) / p->B + 1;
+  if (nb_last > p->m && p->m > 2 && block_gemm_ok(p, Lq, Lk)) {
+    void* bsplit = ws + w.bsplit;
+    uint32_t* bkeys = reinterpret_cast<uint32_t*>(ws + w.bkeys);
+    hsa::launch_ksum_split(ksum, w.nbc * p->d_idx, bsplit, s);
+    if (!hsa::launch_block_score_gemm(q_idx, bsplit, Lq, Lk, p->B, p->m, p->d_idx, w.nbc, bkeys, w.ldb, s)) {
+      *ok = false;
+      return;
+    }
+    hsa::launch_topm_from_keys(rm, Lq, bkeys, w.ldb, p->B, p->m, max_block_candidates(p, Lk), blocks, s);
+  } else {
+    hsa::launch_select_blocks(rm, Lq, q_idx, ksum, 0, p->B, p->m, p->d_idx, blocks,
+                              max_block_candidates(p, Lk), s);
+  }
+}
+
+// Kept tokens for rows [0, Lq) from their kept blocks.
+void run_select_tokens(const hsa_params* p, int64_t Lq, int64_t Lk, const void* q_idx, const void* k_idx,
+                       const int32_t* blocks, int32_t* indices, char* ws, const IndexWs& w, cudaStream_t s,
+                       bool* ok) {
+  hsa::RowMap rm{Lq, Lk, nullptr, 0};
+  if (token_gemm_ok(p, Lq, Lk)) {
+    int* cnt = reinterpret_cast<int*>(ws + w.cnt);
+    int* off = reinterpret_cast<int*>(ws + w.off);
+    int* cursor = reinterpret_cast<int*>(ws + w.cursor);
+    int* ntiles = reinterpret_cast<int*>(ws + w.ntiles);
+    int4* tiles = reinterpret_cast<int4*>(ws + w.tiles);
+    uint32_t* pairs = reinterpret_cast<uint32_t*>(ws + w.pairs);
+    uint32_t* tkeys = reinterpret_cast<uint32_t*>(ws + w.tkeys);
+    hsa::launch_pair_lists(rm, Lq, blocks, p->B, p->m, p->k, int(w.nbins), cnt, off, cursor, tiles, ntiles,
+                           pairs, s);
+    if (!hsa::launch_token_score_gemm(q_idx, k_idx, Lq, Lk, p->B, p->m, p->d_idx, tiles, ntiles, pairs,
+                                      w.max_tiles, tkeys, s)) {
+      *ok = false;
+      return;
+    }
+    hsa::launch_topk_from_keys(rm, Lq, blocks, tkeys, p->B, p->m, p->k, indices, s);
+  } else {
+    hsa::launch_select_tokens(rm, Lq, q_idx, k_idx, blocks, p->B, p->m, p->k, p->d_idx, indices, s);
+  }
+}
+
 
 }  // namespace
 
@@ -128,35 +209,33 @@ int hsa_block_sums(const hsa_params* p, int64_t Lk, const hsa_bf16* k_idx, float
 int hsa_select_blocks(const hsa_params* p, int64_t Lq, int64_t Lk, const hsa_bf16* q_idx,
                       const float* ksum, int32_t* blocks, void* workspace,
                       size_t workspace_bytes, cudaStream_t stream) {
-  (void)workspace;
-  (void)workspace_bytes;
   if (int e = check_index_params(p)) return e;
   if (int e = check_lengths(p, Lq, Lk)) return e;
   if (Lq == 0) return HSA_OK;
   if (!aligned16(q_idx) || !aligned16(blocks) || (Lk / p->B > 0 && !aligned16(ksum)))
     return HSA_ERR_ARG;
+  const IndexWs w = index_ws(p, Lq, Lk);
+  if (!aligned16(workspace) || workspace_bytes < w.total) return HSA_ERR_WORKSPACE;
   if (int e = check_device()) return e;
-  hsa::RowMap rm{Lq, Lk, nullptr, 0};
-  hsa::launch_select_blocks(rm, Lq, q_idx, ksum, 0, p->B, p->m, p->d_idx, blocks,
-                            max_block_candidates(p, Lk), stream);
-  return launch_status();
+  bool ok = true;
+  run_select_blocks(p, Lq, Lk, q_idx, ksum, blocks, static_cast<char*>(workspace), w, stream, &ok);
+  return ok ? launch_status() : HSA_ERR_CUDA;
 }
 
 int hsa_select_tokens(const hsa_params* p, int64_t Lq, int64_t Lk, const hsa_bf16* q_idx,
                       const hsa_bf16* k_idx, const int32_t* blocks, int32_t* indices,
                       void* workspace, size_t workspace_bytes, cudaStream_t stream) {
-  (void)workspace;
-  (void)workspace_bytes;
   if (int e = check_index_params(p)) return e;
   if (int e = check_lengths(p, Lq, Lk)) return e;
   if (Lq == 0) return HSA_OK;
   if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(blocks) || !aligned16(indices))
     return HSA_ERR_ARG;
+  const IndexWs w = index_ws(p, Lq, Lk);
+  if (!aligned16(workspace) || workspace_bytes < w.total) return HSA_ERR_WORKSPACE;
   if (int e = check_device()) return e;
-  hsa::RowMap rm{Lq, Lk, nullptr, 0};
-  hsa::launch_select_tokens(rm, Lq, q_idx, k_idx, blocks, p->B, p->m, p->k, p->d_idx, indices,
-                            stream);
-  return launch_status();
+  bool ok = true;
+  run_select_tokens(p, Lq, Lk, q_idx, k_idx, blocks, indices, static_cast<char*>(workspace), w, stream, &ok);
+  return ok ? launch_status() : HSA_ERR_CUDA;
 }
 
 int hsa_index(const hsa_params* p, int64_t Lq, int64_t Lk, const hsa_bf16* q_idx,
@@ -170,15 +249,13 @@ int hsa_index(const hsa_params* p, int64_t Lq, int64_t Lk, const hsa_bf16* q_idx
   if (!aligned16(workspace) || workspace_bytes < w.total) return HSA_ERR_WORKSPACE;
   if (int e = check_device()) return e;
   char* ws = static_cast<char*>(workspace);
-  float* ksum = reinterpret_cast<float*>(ws + w.ksum_off);
-  int32_t* blocks = reinterpret_cast<int32_t*>(ws + w.blocks_off);
+  float* ksum = reinterpret_cast<float*>(ws + w.ksum);
+  int32_t* blocks = reinterpret_cast<int32_t*>(ws + w.blocks);
+  bool ok = true;
   hsa::launch_block_sums(k_idx, Lk, p->B, p->d_idx, ksum, stream);
-  hsa::RowMap rm{Lq, Lk, nullptr, 0};
-  hsa::launch_select_blocks(rm, Lq, q_idx, ksum, 0, p->B, p->m, p->d_idx, blocks,
-                            max_block_candidates(p, Lk), stream);
-  hsa::launch_select_tokens(rm, Lq, q_idx, k_idx, blocks, p->B, p->m, p->k, p->d_idx, indices,
-                            stream);
-  return launch_status();
+  run_select_blocks(p, Lq, Lk, q_idx, ksum, blocks, ws, w, stream, &ok);
+  if (ok) run_select_tokens(p, Lq, Lk, q_idx, k_idx, blocks, indices, ws, w, stream, &ok);
+  return ok ? launch_status() : HSA_ERR_CUDA;
 }
 
 int hsa_sparse_attn(const hsa_params* p, int64_t Lq, int64_t Lk, const hsa_bf16* Q,

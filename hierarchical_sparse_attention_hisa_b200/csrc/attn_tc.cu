@@ -462,52 +462,12 @@ __global__ void __launch_bounds__(192, 1) sparse_attn_tc_kernel(
   }
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
-                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
-                                  CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      p = nullptr;
-    return reinterpret_cast<EncodeTiledFn>(p);
-  }();
-  return fn;
-}
-
-// 2-D row-major bf16 [rows][cols] map with a {64, box_rows} box, 128B swizzle.
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {64, box_rows};
-  cuuint32_t es[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-int num_sms() {
-  static int n = [] {
-    int dev = 0, v = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-    return v;
-  }();
-  return n;
-}
-
 template <int HP>
 bool launch_hp(const void* Q, const void* K, const void* V, const int32_t* idx, int Lq, int Lk, int k,
                int H, float scale_log2, void* O, cudaStream_t s) {
   CUtensorMap km, vm, qm;
-  if (!make_map(&km, K, uint64_t(Lk), D, 1) || !make_map(&vm, V, uint64_t(Lk), D, 1) ||
-      !make_map(&qm, Q, uint64_t(Lq) * H, D, HP))
+  if (!make_tmap_2d(&km, K, uint64_t(Lk), D, 1) || !make_tmap_2d(&vm, V, uint64_t(Lk), D, 1) ||
+      !make_tmap_2d(&qm, Q, uint64_t(Lq) * H, D, HP))
     return false;
   using C = Cfg<HP>;
   if (cudaFuncSetAttribute(sparse_attn_tc_kernel<HP>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=

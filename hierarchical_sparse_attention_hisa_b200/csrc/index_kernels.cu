@@ -50,6 +50,31 @@ void launch_block_sums(const void* k_idx, int64_t Lk, int B, int d_idx, float* k
 }
 
 // ---------------------------------------------------------------------------
+// Three bf16 planes hi + mid + lo whose sum is the fp32 block sum (the
+// tensor-core block scoring multiplies each plane by bf16 queries; the
+// products are exact and the three partial dot products add up in fp32).
+// ---------------------------------------------------------------------------
+__global__ void ksum_split_kernel(const float* __restrict__ ksum, int64_t n, uint16_t* __restrict__ split) {
+  for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < n; e += int64_t(gridDim.x) * blockDim.x) {
+    const float x = ksum[e];
+    const uint32_t hi = f32_to_bf16_rn(x);
+    const float r1 = x - __uint_as_float(hi << 16);
+    const uint32_t mid = f32_to_bf16_rn(r1);
+    const float r2 = r1 - __uint_as_float(mid << 16);
+    split[e] = uint16_t(hi);
+    split[n + e] = uint16_t(mid);
+    split[2 * n + e] = uint16_t(f32_to_bf16_rn(r2));
+  }
+}
+
+void launch_ksum_split(const float* ksum, int64_t n, void* split, cudaStream_t s) {
+  if (n == 0) return;
+  count_launches(1);
+  const int64_t blocks = (n + 255) / 256;
+  ksum_split_kernel<<<unsigned(blocks < 4096 ? blocks : 4096), 256, 0, s>>>(ksum, n, (uint16_t*)split);
+}
+
+// ---------------------------------------------------------------------------
 // Block selection, one CTA per query row. Candidate c is block c+1 of
 // 1 .. nb-2; its score q . ksum[c+1] is an fp32 dot product (q widened
 // exactly from bf16). The m-2 best candidates by (score desc, block asc) are

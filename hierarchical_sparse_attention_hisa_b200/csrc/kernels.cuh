@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -10,6 +11,11 @@ namespace hsa {
 
 // Counts kernel launches made by this library (see hsa_kernel_launches).
 void count_launches(int n);
+
+// 2-D row-major bf16 [rows][cols] TMA map, box {64 columns, box_rows rows},
+// 128-byte swizzle. False if the driver entry point or the encoding fails.
+bool make_tmap_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+int num_sms();
 
 void launch_block_sums(const void* k_idx, int64_t Lk, int B, int d_idx, float* ksum,
                        cudaStream_t s);
@@ -27,6 +33,19 @@ void launch_sparse_attn_simple(RowMap rm, int64_t rows, const void* Q, const voi
 bool tc_attn_supported(int H, int d, int64_t Lq, int64_t Lk);
 bool launch_sparse_attn_tc(int64_t Lq, const void* Q, const void* K, const void* V, const int32_t* idx,
                            int64_t Lk, int k, int H, float scale, void* O, cudaStream_t s);
+void launch_ksum_split(const float* ksum, int64_t n, void* split, cudaStream_t s);
+bool launch_block_score_gemm(const void* q_idx, const void* bsplit, int64_t Lq, int64_t Lk, int B, int m,
+                             int d_idx, int64_t nbc, uint32_t* out, int64_t ld, cudaStream_t s);
+bool launch_token_score_gemm(const void* q_idx, const void* k_idx, int64_t Lq, int64_t Lk, int B, int m,
+                             int d_idx, const int4* tiles, const int* ntiles, const uint32_t* pairs,
+                             int64_t max_tiles, uint32_t* out, cudaStream_t s);
+void launch_topm_from_keys(RowMap rm, int64_t rows, const uint32_t* bkeys, int64_t ld, int B, int m,
+                           int64_t max_cand, int32_t* blocks, cudaStream_t s);
+void launch_pair_lists(RowMap rm, int64_t rows, const int32_t* blocks, int B, int m, int k, int nbins,
+                       int* cnt, int* off, int* cursor, int4* tiles, int* ntiles, uint32_t* pairs,
+                       cudaStream_t s);
+void launch_topk_from_keys(RowMap rm, int64_t rows, const int32_t* blocks, const uint32_t* tkeys, int B,
+                           int m, int k, int32_t* indices, cudaStream_t s);
 void launch_decode_append(int batch, int64_t capacity, const int32_t* ctx, int B, int d_idx, int d,
                           void* k_idx_cache, void* K_cache, void* V_cache, float* ksum_cache,
                           const void* k_idx_new, const void* K_new, const void* V_new,

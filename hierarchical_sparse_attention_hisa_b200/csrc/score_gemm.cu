@@ -1,0 +1,294 @@
+// Indexer scoring on tcgen05 tensor cores: the two dense contractions of the
+// HISA indexer (page "HISA: Hierarchical Indexed Sparse Attention",
+// sections 第一步 and 第二步), written out as order-preserving uint32 keys
+// for the radix selections that follow.
+//
+//   block scores   S[i][b] = q_idx[i] . ksum[b]     A = 128 query rows (tiled),
+//                  ksum split into three bf16 planes hi + mid + lo (exact for
+//                  |ksum| < 2^24 with at most 24 significant bits), so three
+//                  bf16 MMAs accumulate the fp32 result;
+//   token scores   S[i][s][c] = q_idx[i] . k_idx[b*B + c]   for every (query i,
+//                  slot s) that kept block b: queries that kept the same block
+//                  are gathered (TMA tile::gather4) as the 128 rows of one MMA
+//                  tile against that block's B keys, so each key block is read
+//                  once per 128 queries instead of once per query.
+// Integer-valued inputs make every product and partial sum an exact fp32
+// integer, so the tensor-core results equal the sequential CPU sums.
+//
+// Warp roles of the persistent kernel: warp 0 TMA producer, warp 1 MMA issuer
+// (+ TMEM owner), warps 2-5 epilogue (TMEM -> keys -> global), with a
+// two-deep TMEM accumulator so the epilogue of one tile overlaps the MMAs of
+// the next.
+#include "kernels.cuh"
+#include "tc.cuh"
+
+namespace hsa {
+
+__device__ int g_score_err;
+
+namespace {
+
+using namespace tc;
+
+HSA_DEV bool sg_wait(uint64_t* bar, uint32_t parity, bool& dead) {
+  if (dead) return false;
+  for (uint32_t it = 0; it < (1u << 24); ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 4095u) == 4095u && *(volatile int*)&g_score_err) { dead = true; return false; }
+  }
+  atomicExch(&g_score_err, 1);
+  dead = true;
+  return false;
+}
+HSA_DEV bool sg_wait_warp(uint64_t* bar, uint32_t parity, bool& dead) {
+  bool ok = false;
+  if ((threadIdx.x & 31) == 0) ok = sg_wait(bar, parity, dead);
+  ok = __shfl_sync(kFull, ok ? 1 : 0, 0) != 0;
+  __syncwarp();
+  dead = !ok;
+  return ok;
+}
+
+template <int DK, int N, int NSPLIT>
+struct SG {
+  static constexpr int KB = DK / 64;                 // 128-byte column blocks per row
+  static constexpr int A_BYTES = 128 * DK * 2;
+  static constexpr int B_BYTES = NSPLIT * N * DK * 2;
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int NS = (200 * 1024) / STAGE > 4 ? 4 : (200 * 1024) / STAGE;
+  static constexpr int SMEM = NS * STAGE + 1024;
+  static constexpr int TMEM_COLS = 2 * N < 32 ? 32 : 2 * N;
+};
+
+// Tile source description shared by the roles.
+struct TileArgs {
+  // gathered mode (token scores)
+  const int4* tiles;        // (block, first pair, pair count, -)
+  const int* ntiles;        // device count of tiles
+  const uint32_t* pairs;    // pair = row * m + slot
+  int m, Bsz;
+  // tiled mode (block scores)
+  int Lq, Lk, nb_tiles, m_tiles, nbc;
+  // output
+  uint32_t* out;
+  int64_t ld;
+};
+
+// Tiled mode: does tile (mt, nt) hold any candidate block of any of its rows?
+HSA_DEV bool block_tile_needed(const TileArgs& a, int mt, int nt, int N) {
+  const int last_row = min(a.Lq - 1, mt * 128 + 127);
+  const int64_t t_last = int64_t(a.Lk) - a.Lq + last_row;
+  const int64_t nb_last = t_last / a.Bsz + 1;
+  if (nb_last <= a.m) return false;            // every row keeps all its blocks
+  return int64_t(nt) * N <= nb_last - 2;       // candidates are blocks 1 .. nb-2
+}
+
+template <int DK, int N, int NSPLIT, bool GATHER>
+__global__ void __launch_bounds__(192, 1) score_gemm_kernel(const __grid_constant__ CUtensorMap amap,
+                                                            const __grid_constant__ CUtensorMap bmap,
+                                                            TileArgs ta) {
+  using C = SG<DK, N, NSPLIT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t full[C::NS], empty[C::NS], tfull[2], tempty[2], done;
+  __shared__ uint32_t tmem_base;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::NS; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], 4); }
+    mbar_init(&done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) { tmem_alloc(&tmem_base, C::TMEM_COLS); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+  const int total = GATHER ? *ta.ntiles : ta.m_tiles * ta.nb_tiles;
+  bool dead = false;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) { prefetch_tmap(&amap); prefetch_tmap(&bmap); }
+    uint32_t it = 0;
+    for (int t = blockIdx.x; t < total && !dead; t += gridDim.x) {
+      int a_row0 = 0, b_row0 = 0, rows[4] = {0, 0, 0, 0};
+      if (GATHER) {
+        const int4 d = ta.tiles[t];
+        b_row0 = d.x * ta.Bsz;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int r = lane * 4 + e;
+          rows[e] = r < d.z ? int(ta.pairs[d.y + r] / uint32_t(ta.m)) : 0;
+        }
+      } else {
+        const int mt = t / ta.nb_tiles, nt = t % ta.nb_tiles;
+        if (!block_tile_needed(ta, mt, nt, N)) continue;
+        a_row0 = mt * 128;
+        b_row0 = nt * N;
+      }
+      const int s = it % C::NS;
+      if (!sg_wait_warp(&empty[s], ((it / C::NS) & 1) ^ 1, dead)) break;
+      uint8_t* a_s = sm + s * C::STAGE;
+      uint8_t* b_s = a_s + C::A_BYTES;
+      if (lane == 0) mbar_arrive_expect_tx(&full[s], C::STAGE);
+      __syncwarp();
+      if (GATHER) {
+#pragma unroll
+        for (int kb = 0; kb < C::KB; ++kb)
+          tma_gather4(a_s + kb * 128 * 128 + lane * 512, &amap, &full[s], kb * 64, rows[0], rows[1], rows[2], rows[3]);
+      } else if (lane == 0) {
+#pragma unroll
+        for (int kb = 0; kb < C::KB; ++kb) tma_load_2d(a_s + kb * 128 * 128, &amap, &full[s], kb * 64, a_row0);
+      }
+      if (lane == 0) {
+#pragma unroll
+        for (int sp = 0; sp < NSPLIT; ++sp)
+#pragma unroll
+          for (int kb = 0; kb < C::KB; ++kb)
+            tma_load_2d(b_s + sp * N * DK * 2 + kb * N * 128, &bmap, &full[s], kb * 64,
+                        b_row0 + sp * ta.nbc);
+      }
+      ++it;
+    }
+    if (lane == 0) {  // drain armed loads
+      bool d2 = false;
+      for (uint32_t u = (it >= uint32_t(C::NS) ? it - C::NS : 0); u < it; ++u)
+        sg_wait(&full[u % C::NS], (u / C::NS) & 1, d2);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(128, N, false, false);
+      uint32_t it = 0;
+      for (int t = blockIdx.x; t < total && !dead; t += gridDim.x) {
+        if (!GATHER && !block_tile_needed(ta, t / ta.nb_tiles, t % ta.nb_tiles, N)) continue;
+        const int s = it % C::NS, tb = it & 1;
+        if (!sg_wait(&full[s], (it / C::NS) & 1, dead)) break;
+        if (!sg_wait(&tempty[tb], ((it >> 1) & 1) ^ 1, dead)) break;
+        tc_fence_after();
+        const uint32_t a_s = smem_u32(sm + s * C::STAGE);
+        const uint32_t b_s = a_s + C::A_BYTES;
+        uint32_t acc = 0;
+#pragma unroll
+        for (int sp = 0; sp < NSPLIT; ++sp)
+#pragma unroll
+          for (int ks = 0; ks < DK / 16; ++ks) {
+            const uint64_t a = smem_desc(a_s + (ks / 4) * 128 * 128 + (ks % 4) * 32, 16, 1024, kSw128);
+            const uint64_t b = smem_desc(b_s + sp * N * DK * 2 + (ks / 4) * N * 128 + (ks % 4) * 32, 16, 1024, kSw128);
+            mma_bf16(tmem + tb * N, a, b, idesc, acc);
+            acc = 1;
+          }
+        mma_commit(&empty[s]);
+        mma_commit(&tfull[tb]);
+        ++it;
+      }
+      mma_commit(&done);
+      bool d2 = false;
+      sg_wait(&done, 0, d2);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quad = warp & 3, r = quad * 32 + lane;
+    const uint32_t lane_addr = uint32_t(quad * 32) << 16;
+    uint32_t it = 0;
+    for (int t = blockIdx.x; t < total && !dead; t += gridDim.x) {
+      uint32_t* dst = nullptr;
+      if (GATHER) {
+        const int4 d = ta.tiles[t];
+        if (r < d.z) dst = ta.out + int64_t(ta.pairs[d.y + r]) * ta.ld;
+      } else {
+        const int mt = t / ta.nb_tiles, nt = t % ta.nb_tiles;
+        if (!block_tile_needed(ta, mt, nt, N)) continue;
+        const int row = mt * 128 + r;
+        if (row < ta.Lq) dst = ta.out + int64_t(row) * ta.ld + int64_t(nt) * N;
+      }
+      const int tb = it & 1;
+      if (!sg_wait_warp(&tfull[tb], (it >> 1) & 1, dead)) break;
+      tc_fence_after();
+#pragma unroll 2
+      for (int c0 = 0; c0 < N; c0 += 16) {
+        uint32_t v[16];
+        tmem_ld16(tmem + lane_addr + tb * N + c0, v);
+        tmem_wait_ld();
+        if (dst) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            d4[e] = make_uint4(score_key(__uint_as_float(v[4 * e])), score_key(__uint_as_float(v[4 * e + 1])),
+                               score_key(__uint_as_float(v[4 * e + 2])), score_key(__uint_as_float(v[4 * e + 3])));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[tb]);
+      ++it;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int DK, int N, int NSPLIT, bool GATHER>
+bool launch_sg(const CUtensorMap& am, const CUtensorMap& bm, const TileArgs& ta, int grid, cudaStream_t s) {
+  using C = SG<DK, N, NSPLIT>;
+  auto kern = score_gemm_kernel<DK, N, NSPLIT, GATHER>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess) return false;
+  kern<<<grid, 192, C::SMEM, s>>>(am, bm, ta);
+  count_launches(1);
+  return true;
+}
+
+}  // namespace
+
+// Block scores for rows [0, Lq): out[i][b] = key(q_idx[i] . ksum[b]) for the
+// tiles that hold candidate blocks (others are left unwritten).
+// bsplit: [3][nbc][d_idx] bf16 planes hi, mid, lo of ksum.
+bool launch_block_score_gemm(const void* q_idx, const void* bsplit, int64_t Lq, int64_t Lk, int B, int m,
+                             int d_idx, int64_t nbc, uint32_t* out, int64_t ld, cudaStream_t s) {
+  constexpr int N = 64;
+  CUtensorMap am, bm;
+  if (!make_tmap_2d(&am, q_idx, uint64_t(Lq), uint64_t(d_idx), 128) ||
+      !make_tmap_2d(&bm, bsplit, uint64_t(3 * nbc), uint64_t(d_idx), N))
+    return false;
+  TileArgs ta{};
+  ta.m = m; ta.Bsz = B; ta.Lq = int(Lq); ta.Lk = int(Lk); ta.nbc = int(nbc);
+  ta.m_tiles = int((Lq + 127) / 128);
+  ta.nb_tiles = int((nbc + N - 1) / N);
+  ta.out = out; ta.ld = ld;
+  const int64_t tiles = int64_t(ta.m_tiles) * ta.nb_tiles;
+  const int grid = int(tiles < num_sms() ? tiles : num_sms());
+  if (grid == 0) return true;
+  if (d_idx == 128) return launch_sg<128, N, 3, false>(am, bm, ta, grid, s);
+  return launch_sg<64, N, 3, false>(am, bm, ta, grid, s);
+}
+
+// Token scores for the (row, slot) pairs listed per key block:
+// out[pair][c] = key(q_idx[pair / m] . k_idx[block * B + c]), c < B.
+bool launch_token_score_gemm(const void* q_idx, const void* k_idx, int64_t Lq, int64_t Lk, int B, int m,
+                             int d_idx, const int4* tiles, const int* ntiles, const uint32_t* pairs,
+                             int64_t max_tiles, uint32_t* out, cudaStream_t s) {
+  CUtensorMap am, bm;
+  if (!make_tmap_2d(&am, q_idx, uint64_t(Lq), uint64_t(d_idx), 1) ||
+      !make_tmap_2d(&bm, k_idx, uint64_t(Lk), uint64_t(d_idx), B))
+    return false;
+  TileArgs ta{};
+  ta.tiles = tiles; ta.ntiles = ntiles; ta.pairs = pairs; ta.m = m; ta.Bsz = B;
+  ta.out = out; ta.ld = B;
+  const int grid = int(max_tiles < num_sms() ? (max_tiles > 0 ? max_tiles : 1) : num_sms());
+  if (d_idx == 128) {
+    if (B == 128) return launch_sg<128, 128, 1, true>(am, bm, ta, grid, s);
+    if (B == 64) return launch_sg<128, 64, 1, true>(am, bm, ta, grid, s);
+  } else {
+    if (B == 128) return launch_sg<64, 128, 1, true>(am, bm, ta, grid, s);
+    if (B == 64) return launch_sg<64, 64, 1, true>(am, bm, ta, grid, s);
+  }
+  return false;
+}
+
+}  // namespace hsa

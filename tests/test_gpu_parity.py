@@ -61,10 +61,19 @@ def test_select_blocks_bit_exact(hsa, Lq, Lk, B, m, d):
     ks = torch.empty((max(Lk // B, 1), d), dtype=torch.float32, device="cuda")
     hsa.hsa_block_sums(p, Lk, dev(k), ks)
     blocks = torch.empty((Lq, m), dtype=torch.int32, device="cuda")
-    hsa.hsa_select_blocks(p, Lq, Lk, dev(q), ks, blocks)
+    ws = torch.empty(hsa.hsa_index_workspace_size(p, Lq, Lk), dtype=torch.uint8, device="cuda")
+    hsa.hsa_select_blocks(p, Lq, Lk, dev(q), ks, blocks, ws)
     torch.cuda.synchronize()
     want = oracle.select_blocks(q, oracle.block_sums(k, B), Lk, B, m)
     assert np.array_equal(blocks.cpu().numpy(), want)
+    # token stage on the same blocks, through its own entry point
+    kk = 3 * B
+    p.k = kk
+    ws = torch.empty(hsa.hsa_index_workspace_size(p, Lq, Lk), dtype=torch.uint8, device="cuda")
+    idx = torch.empty((Lq, kk), dtype=torch.int32, device="cuda")
+    hsa.hsa_select_tokens(p, Lq, Lk, dev(q), dev(k), blocks, idx, ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(idx.cpu().numpy(), oracle.select_tokens(q, k, want, B, kk))
 
 
 # ------------------------------------------------------------------ indexer
@@ -93,6 +102,9 @@ def test_index_prefill_16k_all_rows(hsa):
     (600, 600, 32, 4, 1, 64),         # k = 1
     (400, 400, 8, 5, 40, 128),        # k = m*B: every candidate of a full row kept
     (333, 1000, 10, 12, 100, 64),     # B not a power of two
+    (3000, 9000, 64, 16, 300, 128),   # tensor-core path, B = 64, chunk of queries
+    (2500, 2500, 64, 10, 200, 64),    # tensor-core path, d_idx = 64
+    (129, 20000, 128, 24, 1000, 128), # one M tile plus one row
 ])
 def test_index_shapes_bit_exact(hsa, Lq, Lk, B, m, k, d):
     q, kk = synth.int_bf16((Lq, d), 13, 1), synth.int_bf16((Lk, d), 13, 2)
