@@ -33,9 +33,11 @@ constexpr int D = 128;       // head dim handled by this kernel
 constexpr int TILE = 128;    // kept keys per MMA tile (the M dimension)
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
-template <int HP>
+template <int HP, int NPW>
 struct Cfg {
   static constexpr int NS = HP <= 32 ? 3 : 2;       // K/V pipeline stages
+  static constexpr int HH = HP / 2;                 // heads per softmax warpgroup
+  static constexpr int NWARPS = NPW + 1 + 8;        // producers, MMA issuer, 2 softmax warpgroups
   static constexpr int KV_BYTES = TILE * D * 2;     // one K or V tile: 32 KB
   static constexpr int Q_BYTES = HP * D * 2;        // one query's heads
   static constexpr int P_ROW = HP * 2;              // bytes of one P^T row (<= 128)
@@ -52,7 +54,7 @@ struct Cfg {
 struct Bars {
   uint64_t kfull[3], kempty[3], vfull[3], vempty[3];
   uint64_t qfull[2], qempty[2], sfull[2], sempty[2], pfull[2], pempty[2], ofull[2], oempty[2];
-  uint64_t done, group;
+  uint64_t done, group[2];
 };
 
 // Bounded wait that also gives up as soon as another role has reported a
@@ -131,12 +133,51 @@ HSA_DEV int transpose_head(int lane, int i) {
   return lane >> shift;
 }
 
-template <int HP>
-__global__ void __launch_bounds__(192, 1) sparse_attn_tc_kernel(
-    const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
-    const __grid_constant__ CUtensorMap qmap, const int32_t* __restrict__ idx, int Lq, int Lk, int k,
-    int H, float scale_log2, uint16_t* __restrict__ O) {
-  using C = Cfg<HP>;
+// HH consecutive TMEM columns of this warp's 32 lanes into v (HH = 8, 16 or 32).
+template <int HH>
+HSA_DEV void tmem_ld_cols(uint32_t taddr, float (&v)[HH]) {
+  if constexpr (HH == 8) {
+    uint32_t r[8];
+    tmem_ld8(taddr, r);
+    tmem_wait_ld();
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(r[e]);
+  } else {
+#pragma unroll
+    for (int c0 = 0; c0 < HH; c0 += 16) {
+      uint32_t r[16];
+      tmem_ld16(taddr + c0, r);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 16; ++e) v[c0 + e] = __uint_as_float(r[e]);
+    }
+  }
+}
+template <int HH>
+HSA_DEV void tmem_st_cols(uint32_t taddr, const float (&v)[HH]) {
+  if constexpr (HH == 8) {
+    uint32_t r[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) r[e] = __float_as_uint(v[e]);
+    tmem_st8(taddr, r);
+  } else {
+#pragma unroll
+    for (int c0 = 0; c0 < HH; c0 += 16) {
+      uint32_t r[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(v[c0 + e]);
+      tmem_st16(taddr + c0, r);
+    }
+  }
+  tmem_wait_st();
+}
+
+template <int HP, int NPW>
+__global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_kernel(
+    const __grid_constant__ CUtensorMap qmap, const uint16_t* __restrict__ K, const uint16_t* __restrict__ V,
+    const int32_t* __restrict__ idx, int Lq, int Lk, int k, int H, float scale_log2, uint16_t* __restrict__ O) {
+  using C = Cfg<HP, NPW>;
+  constexpr int HH = C::HH;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ __align__(8) Bars bars;
@@ -145,39 +186,42 @@ __global__ void __launch_bounds__(192, 1) sparse_attn_tc_kernel(
   __shared__ float red[4][HP];
   __shared__ float mh[HP];
   __shared__ float lsum[HP];
-  __shared__ int vote[2][4];
+  __shared__ int vote[2][2][4];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NS; ++s) {
-      mbar_init(&bars.kfull[s], 1); mbar_init(&bars.kempty[s], 1);
-      mbar_init(&bars.vfull[s], 1); mbar_init(&bars.vempty[s], 1);
+      mbar_init(&bars.kfull[s], NPW * 32); mbar_init(&bars.kempty[s], 1);
+      mbar_init(&bars.vfull[s], NPW * 32); mbar_init(&bars.vempty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&bars.qfull[b], 1); mbar_init(&bars.qempty[b], 1 + 4);
-      mbar_init(&bars.sfull[b], 1); mbar_init(&bars.sempty[b], 4);
-      mbar_init(&bars.pfull[b], 4); mbar_init(&bars.pempty[b], 1);
-      mbar_init(&bars.ofull[b], 1); mbar_init(&bars.oempty[b], 4);
+      mbar_init(&bars.qfull[b], 1); mbar_init(&bars.qempty[b], 1 + 8);
+      mbar_init(&bars.sfull[b], 1); mbar_init(&bars.sempty[b], 8);
+      mbar_init(&bars.pfull[b], 8); mbar_init(&bars.pempty[b], 1);
+      mbar_init(&bars.ofull[b], 1); mbar_init(&bars.oempty[b], 8);
+      mbar_init(&bars.group[b], 4);
     }
     mbar_init(&bars.done, 1);
-    mbar_init(&bars.group, 4);
     fence_barrier_init();
   }
-  if (warp == 1) { tmem_alloc(&tmem_base, C::TMEM_COLS); tmem_relinquish(); }
+  if (warp == NPW) { tmem_alloc(&tmem_base, C::TMEM_COLS); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base;
   bool dead = false;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) { prefetch_tmap(&kmap); prefetch_tmap(&vmap); prefetch_tmap(&qmap); }
+  if (warp < NPW) {
+    // ------------------------------------------------------------ producers
+    // Producer thread p copies the (row, 16-byte chunk) pairs p, p + 32*NPW, ...
+    // of each K and V tile with cp.async into the 128B-swizzled layout UMMA reads.
+    constexpr int PT = NPW * 32, PER = (TILE * 16 + PT - 1) / PT;
+    const int p = threadIdx.x;
+    if (p == 0) prefetch_tmap(&qmap);
     uint32_t g = 0, qn = 0;
     for (int q = blockIdx.x; q < Lq && !dead; q += gridDim.x, ++qn) {
       const int32_t* row = idx + int64_t(q) * k;
-      // tiles = ceil((last valid position + 1) / TILE)
-      int last = -1;
+      int last = -1;  // tiles = ceil((last valid position + 1) / TILE)
       if ((k & 3) == 0) {
         const int4* row4 = reinterpret_cast<const int4*>(row);
 #pragma unroll 4
@@ -189,57 +233,58 @@ __global__ void __launch_bounds__(192, 1) sparse_attn_tc_kernel(
           if (v.w >= 0 && v.w < Lk) last = 4 * p4 + 3;
         }
       } else {
-        for (int p = lane; p < k; p += 32) {
-          const int j = __ldg(row + p);
-          if (j >= 0 && j < Lk) last = p;
+        for (int pp = lane; pp < k; pp += 32) {
+          const int j = __ldg(row + pp);
+          if (j >= 0 && j < Lk) last = pp;
         }
       }
 #pragma unroll
       for (int o = 16; o >= 1; o >>= 1) last = max(last, __shfl_xor_sync(kFull, last, o));
       const int nt = (last + TILE) / TILE;
       const int qb = qn & 1;
-      if (!wait_warp(&bars.qempty[qb], ((qn >> 1) & 1) ^ 1, dead)) break;
-      if (lane == 0) {
-        qinfo[qb] = nt;
-        mbar_arrive_expect_tx(&bars.qfull[qb], C::Q_BYTES);
-        uint8_t* qt = sm + C::OFF_Q + qb * C::Q_BYTES;
-        tma_load_2d(qt, &qmap, &bars.qfull[qb], 0, q * H);
-        tma_load_2d(qt + HP * 128, &qmap, &bars.qfull[qb], 64, q * H);
+      if (warp == 0) {
+        if (!wait_warp(&bars.qempty[qb], ((qn >> 1) & 1) ^ 1, dead)) break;
+        if (lane == 0) {
+          qinfo[qb] = nt;
+          mbar_arrive_expect_tx(&bars.qfull[qb], C::Q_BYTES);
+          uint8_t* qt = sm + C::OFF_Q + qb * C::Q_BYTES;
+          tma_load_2d(qt, &qmap, &bars.qfull[qb], 0, q * H);
+          tma_load_2d(qt + HP * 128, &qmap, &bars.qfull[qb], 64, q * H);
+        }
       }
       for (int i = 0; i < nt && !dead; ++i, ++g) {
         const int s = g % C::NS;
         const uint32_t ph = (g / C::NS) & 1;
-        int r4[4];
+        int64_t src[PER];
+        uint32_t dst[PER];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int p = i * TILE + lane * 4 + e;
-          const int j = p < k ? __ldg(row + p) : -1;
-          r4[e] = (j >= 0 && j < Lk) ? j : 0;
+        for (int u = 0; u < PER; ++u) {
+          const int e = p + u * PT, r = (e >> 4) & (TILE - 1), c = e & 15;
+          const int pos = i * TILE + r;
+          const int j = (e < TILE * 16 && pos < k) ? __ldg(row + pos) : -1;
+          src[u] = int64_t((j >= 0 && j < Lk) ? j : 0) * D + c * 8;
+          dst[u] = (c >> 3) * (TILE * 128) + swz_offset(r, c & 7, 128);
         }
         if (!wait_warp(&bars.kempty[s], ph ^ 1, dead)) break;
-        if (lane == 0) mbar_arrive_expect_tx(&bars.kfull[s], C::KV_BYTES);
-        __syncwarp();
-        uint8_t* kt = sm + C::OFF_K + s * C::KV_BYTES + lane * 4 * 128;
-        tma_gather4(kt, &kmap, &bars.kfull[s], 0, r4[0], r4[1], r4[2], r4[3]);
-        tma_gather4(kt + TILE * 128, &kmap, &bars.kfull[s], 64, r4[0], r4[1], r4[2], r4[3]);
+        const uint32_t kt = smem_u32(sm + C::OFF_K + s * C::KV_BYTES);
+#pragma unroll
+        for (int u = 0; u < PER; ++u)
+          if (p + u * PT < TILE * 16) cp_async16(kt + dst[u], K + src[u]);
+        cp_async_arrive(&bars.kfull[s]);
         if (!wait_warp(&bars.vempty[s], ph ^ 1, dead)) break;
-        if (lane == 0) mbar_arrive_expect_tx(&bars.vfull[s], C::KV_BYTES);
-        __syncwarp();
-        uint8_t* vt = sm + C::OFF_V + s * C::KV_BYTES + lane * 4 * 128;
-        tma_gather4(vt, &vmap, &bars.vfull[s], 0, r4[0], r4[1], r4[2], r4[3]);
-        tma_gather4(vt + TILE * 128, &vmap, &bars.vfull[s], 64, r4[0], r4[1], r4[2], r4[3]);
+        const uint32_t vt = smem_u32(sm + C::OFF_V + s * C::KV_BYTES);
+#pragma unroll
+        for (int u = 0; u < PER; ++u)
+          if (p + u * PT < TILE * 16) cp_async16(vt + dst[u], V + src[u]);
+        cp_async_arrive(&bars.vfull[s]);
       }
     }
-    // Drain: every armed load has landed before the CTA may exit.
-    if (lane == 0) {
+    cp_async_wait_all();  // every copy has landed before the CTA may exit
+    if (warp == 0 && lane == 0) {
       bool d2 = false;
-      for (uint32_t t = (g >= uint32_t(C::NS) ? g - C::NS : 0); t < g; ++t) {
-        wait_bar(&bars.kfull[t % C::NS], (t / C::NS) & 1, d2);
-        wait_bar(&bars.vfull[t % C::NS], (t / C::NS) & 1, d2);
-      }
       for (uint32_t t = (qn >= 2 ? qn - 2 : 0); t < qn; ++t) wait_bar(&bars.qfull[t & 1], (t >> 1) & 1, d2);
     }
-  } else if (warp == 1) {
+  } else if (warp == NPW) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_bf16(128, HP, false, false);
@@ -292,18 +337,20 @@ __global__ void __launch_bounds__(192, 1) sparse_attn_tc_kernel(
         ++oq;
       }
       if (prev.valid && !dead) issue_pv(prev);
-      // all issued MMAs complete before TMEM is released
-      mma_commit(&bars.done);
+      mma_commit(&bars.done);  // all issued MMAs complete before TMEM is released
       bool d2 = false;
       wait_bar(&bars.done, 0, d2);
     }
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax / epilogue
+    // Two warpgroups; warpgroup wg owns heads [wg*HH, wg*HH + HH) of every tile.
+    const int sw = warp - NPW - 1, wg = sw >> 2, wq = sw & 3;
     const int quad = warp & 3;              // TMEM lane quadrant this warp may access
     const int r = quad * 32 + lane;         // key row of the tile / dim row of O^T
+    const int h0 = wg * HH;                 // first head of this warpgroup
     const uint32_t lane_addr = uint32_t(quad * 32) << 16;
-    const int wq = warp - 2;                // 0..3 index among softmax warps
+    uint64_t* gbar = &bars.group[wg];
     uint32_t g = 0, qn = 0, oq = 0, gph = 0;
     for (int q = blockIdx.x; q < Lq && !dead; q += gridDim.x, ++qn) {
       const int qb = qn & 1;
@@ -313,35 +360,28 @@ __global__ void __launch_bounds__(192, 1) sparse_attn_tc_kernel(
       if (lane == 0) mbar_arrive(&bars.qempty[qb]);
       uint16_t* orow = O + int64_t(q) * H * D;
       if (nt == 0) {
-        for (int h = 0; h < H; ++h) orow[h * D + r] = 0;
+        for (int h = h0; h < h0 + HH && h < H; ++h) orow[h * D + r] = 0;
         continue;
       }
       const uint32_t ob = oq & 1;
       const int32_t* irow = idx + int64_t(q) * k;
-      float lp[HP];
+      float lp[HH];
 #pragma unroll
-      for (int h = 0; h < HP; ++h) lp[h] = 0.f;
+      for (int h = 0; h < HH; ++h) lp[h] = 0.f;
       for (int i = 0; i < nt && !dead; ++i, ++g) {
         const int sb = g & 1;
-        const int p = i * TILE + r;
-        const int j = p < k ? __ldg(irow + p) : -1;
+        const int pos = i * TILE + r;
+        const int j = pos < k ? __ldg(irow + pos) : -1;
         const bool valid = j >= 0 && j < Lk;
         if (!wait_warp(&bars.sfull[sb], (g >> 1) & 1, dead)) break;
         tc_fence_after();
-        float x[HP];
-#pragma unroll
-        for (int c0 = 0; c0 < HP; c0 += 16) {
-          uint32_t v[16];
-          tmem_ld16(tmem + lane_addr + sb * HP + c0, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 16; ++e) x[c0 + e] = __uint_as_float(v[e]);
-        }
+        float x[HH];
+        tmem_ld_cols<HH>(tmem + lane_addr + sb * HP + h0, x);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.sempty[sb]);
 #pragma unroll
-        for (int h = 0; h < HP; ++h) x[h] = (valid && h < H) ? x[h] * scale_log2 : -INFINITY;
+        for (int h = 0; h < HH; ++h) x[h] = (valid && h0 + h < H) ? x[h] * scale_log2 : -INFINITY;
 
         // Raise the running maxima only on the first tile, or when some
         // score exceeds its head's maximum by more than the threshold.
@@ -349,70 +389,66 @@ __global__ void __launch_bounds__(192, 1) sparse_attn_tc_kernel(
         if (!need_max) {
           bool mine = false;
 #pragma unroll
-          for (int h = 0; h < HP; ++h) mine |= x[h] > mh[h] + kRescaleThreshold;
+          for (int h = 0; h < HH; ++h) mine |= x[h] > mh[h0 + h] + kRescaleThreshold;
           const bool any = __any_sync(kFull, mine);
-          if (lane == 0) vote[gph & 1][wq] = any;
           const uint32_t vb = gph & 1;
-          if (!group_sync(&bars.group, gph, dead)) break;
-          need_max = vote[vb][0] | vote[vb][1] | vote[vb][2] | vote[vb][3];
+          if (lane == 0) vote[vb][wg][wq] = any;
+          if (!group_sync(gbar, gph, dead)) break;
+          need_max = vote[vb][wg][0] | vote[vb][wg][1] | vote[vb][wg][2] | vote[vb][wg][3];
         }
         if (need_max) {
 #pragma unroll
-          for (int h = 0; h < HP; ++h) {
+          for (int h = 0; h < HH; ++h) {
             const float wm = redux_max(x[h]);
-            if (lane == (h & 31)) red[wq][h] = wm;
+            if (lane == (h & 31)) red[wq][h0 + h] = wm;
           }
-          if (!group_sync(&bars.group, gph, dead)) break;
-          if (r < HP) {
-            const float tm = fmaxf(fmaxf(red[0][r], red[1][r]), fmaxf(red[2][r], red[3][r]));
-            const float old = i == 0 ? -INFINITY : mh[r];
-            red[0][r] = old;  // the previous maximum, for the rescale factors
-            mh[r] = fmaxf(old, tm);
+          if (!group_sync(gbar, gph, dead)) break;
+          if (r < HH) {
+            const int hh = h0 + r;
+            const float tm = fmaxf(fmaxf(red[0][hh], red[1][hh]), fmaxf(red[2][hh], red[3][hh]));
+            const float old = i == 0 ? -INFINITY : mh[hh];
+            red[0][hh] = old;  // the previous maximum, for the rescale factors
+            mh[hh] = fmaxf(old, tm);
           }
-          if (!group_sync(&bars.group, gph, dead)) break;
+          if (!group_sync(gbar, gph, dead)) break;
           if (i > 0) {
-            // rescale l and the O^T accumulator by 2^(old - new) per head;
+            // rescale l and this warpgroup's O^T columns by 2^(old - new);
             // the previous tile's PV must have landed first.
             const uint32_t pg = g - 1;
             if (!wait_warp(&bars.pempty[pg & 1], (pg >> 1) & 1, dead)) break;
             tc_fence_after();
+            float ov[HH];
+            const uint32_t ta = tmem + lane_addr + 2 * HP + ob * HP + h0;
+            tmem_ld_cols<HH>(ta, ov);
 #pragma unroll
-            for (int c0 = 0; c0 < HP; c0 += 16) {
-              uint32_t v[16];
-              const uint32_t ta = tmem + lane_addr + 2 * HP + ob * HP + c0;
-              tmem_ld16(ta, v);
-              tmem_wait_ld();
-#pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                const float o = red[0][c0 + e], n = mh[c0 + e];
-                const float a = (o == -INFINITY || n == -INFINITY) ? (o == n ? 1.f : 0.f) : exp2f(o - n);
-                lp[c0 + e] *= a;
-                v[e] = __float_as_uint(__uint_as_float(v[e]) * a);
-              }
-              tmem_st16(ta, v);
+            for (int h = 0; h < HH; ++h) {
+              const float o = red[0][h0 + h], n = mh[h0 + h];
+              const float a = (o == -INFINITY || n == -INFINITY) ? (o == n ? 1.f : 0.f) : exp2f(o - n);
+              lp[h] *= a;
+              ov[h] *= a;
             }
-            tmem_wait_st();
+            tmem_st_cols<HH>(ta, ov);
             // red[0] holds the old maxima until every thread has read them
-            if (!group_sync(&bars.group, gph, dead)) break;
+            if (!group_sync(gbar, gph, dead)) break;
           }
         }
-        // probabilities, partial row sums, P^T row into smem (bf16, swizzled)
+        // probabilities, partial row sums, this warpgroup's part of the P^T row
         const int pb = g & 1;
         if (!wait_warp(&bars.pempty[pb], ((g >> 1) & 1) ^ 1, dead)) break;
         uint8_t* prow = sm + C::OFF_P + pb * C::P_BYTES;
 #pragma unroll
-        for (int c = 0; c < HP / 8; ++c) {
+        for (int c = 0; c < HH / 8; ++c) {
           uint32_t w[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int h0 = c * 8 + 2 * e;
-            const float p0 = x[h0] == -INFINITY ? 0.f : exp2f(x[h0] - mh[h0]);
-            const float p1 = x[h0 + 1] == -INFINITY ? 0.f : exp2f(x[h0 + 1] - mh[h0 + 1]);
-            lp[h0] += p0;
-            lp[h0 + 1] += p1;
+            const int a0 = c * 8 + 2 * e;
+            const float p0 = x[a0] == -INFINITY ? 0.f : exp2f(x[a0] - mh[h0 + a0]);
+            const float p1 = x[a0 + 1] == -INFINITY ? 0.f : exp2f(x[a0 + 1] - mh[h0 + a0 + 1]);
+            lp[a0] += p0;
+            lp[a0 + 1] += p1;
             w[e] = pack_bf16x2(p0, p1);
           }
-          *reinterpret_cast<uint4*>(prow + swz_offset(r, c, C::P_ROW)) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(prow + swz_offset(r, h0 / 8 + c, C::P_ROW)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -420,62 +456,59 @@ __global__ void __launch_bounds__(192, 1) sparse_attn_tc_kernel(
         if (lane == 0) mbar_arrive(&bars.pfull[pb]);
       }
       if (dead) break;
-      // ---- epilogue: row sums, normalise O^T, write O[q][h][r]
-      warp_transpose_sum<HP>(lp);
-      constexpr int NL = HP >= 32 ? HP / 32 : 1;
-      if (HP >= 32 || (lane & ((32 / HP) - 1)) == 0) {
+      // ---- epilogue: row sums, normalise O^T, write O[q][h][r] for this warpgroup's heads
+      warp_transpose_sum<HH>(lp);
+      constexpr int NL = HH >= 32 ? HH / 32 : 1;
+      if (HH >= 32 || (lane & ((32 / HH) - 1)) == 0) {
 #pragma unroll
-        for (int e = 0; e < NL; ++e) red[wq][transpose_head<HP>(lane, e)] = lp[e];
+        for (int e = 0; e < NL; ++e) red[wq][h0 + transpose_head<HH>(lane, e)] = lp[e];
       }
-      if (!group_sync(&bars.group, gph, dead)) break;
-      if (r < HP) lsum[r] = red[0][r] + red[1][r] + red[2][r] + red[3][r];
-      if (!group_sync(&bars.group, gph, dead)) break;
+      if (!group_sync(gbar, gph, dead)) break;
+      if (r < HH) lsum[h0 + r] = red[0][h0 + r] + red[1][h0 + r] + red[2][h0 + r] + red[3][h0 + r];
+      if (!group_sync(gbar, gph, dead)) break;
       if (!wait_warp(&bars.ofull[ob], (oq >> 1) & 1, dead)) break;
       tc_fence_after();
+      float ov[HH];
+      tmem_ld_cols<HH>(tmem + lane_addr + 2 * HP + ob * HP + h0, ov);
 #pragma unroll
-      for (int c0 = 0; c0 < HP; c0 += 16) {
-        uint32_t v[16];
-        tmem_ld16(tmem + lane_addr + 2 * HP + ob * HP + c0, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int h = c0 + e;
-          if (h < H) {
-            const float l = lsum[h];
-            orow[h * D + r] = uint16_t(f32_to_bf16_rn(l > 0.f ? __uint_as_float(v[e]) / l : 0.f));
-          }
+      for (int h = 0; h < HH; ++h) {
+        if (h0 + h < H) {
+          const float l = lsum[h0 + h];
+          orow[(h0 + h) * D + r] = uint16_t(f32_to_bf16_rn(l > 0.f ? ov[h] / l : 0.f));
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.oempty[ob]);
-      // lsum / red are reused by the next query only after everyone is done
-      if (!group_sync(&bars.group, gph, dead)) break;
+      // lsum / red are reused by the next query only after the warpgroup is done
+      if (!group_sync(gbar, gph, dead)) break;
       ++oq;
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == NPW) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
+// 7 producer warps + 1 MMA warp + 8 softmax warps = 16 warps, 4 per SM
+// sub-partition, which leaves 128 registers per thread.
+constexpr int kProducerWarps = 7;
+
 template <int HP>
 bool launch_hp(const void* Q, const void* K, const void* V, const int32_t* idx, int Lq, int Lk, int k,
                int H, float scale_log2, void* O, cudaStream_t s) {
-  CUtensorMap km, vm, qm;
-  if (!make_tmap_2d(&km, K, uint64_t(Lk), D, 1) || !make_tmap_2d(&vm, V, uint64_t(Lk), D, 1) ||
-      !make_tmap_2d(&qm, Q, uint64_t(Lq) * H, D, HP))
-    return false;
-  using C = Cfg<HP>;
-  if (cudaFuncSetAttribute(sparse_attn_tc_kernel<HP>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
-      cudaSuccess)
+  CUtensorMap qm;
+  if (!make_tmap_2d(&qm, Q, uint64_t(Lq) * H, D, HP)) return false;
+  using C = Cfg<HP, kProducerWarps>;
+  auto kern = sparse_attn_tc_kernel<HP, kProducerWarps>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
     return false;
   const int grid = Lq < num_sms() ? Lq : num_sms();
-  sparse_attn_tc_kernel<HP><<<grid, 192, C::SMEM, s>>>(km, vm, qm, idx, Lq, Lk, k, H, scale_log2,
-                                                       static_cast<uint16_t*>(O));
+  kern<<<grid, 32 * C::NWARPS, C::SMEM, s>>>(qm, static_cast<const uint16_t*>(K), static_cast<const uint16_t*>(V),
+                                             idx, Lq, Lk, k, H, scale_log2, static_cast<uint16_t*>(O));
   return true;
 }
 
