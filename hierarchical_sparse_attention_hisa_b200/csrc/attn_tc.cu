@@ -9,15 +9,23 @@
 //                                                  B = the query's H x d block)
 //   O^T[c][h]  += Vtile[key][c] . P^T[key][h]     (A = gathered V rows read
 //                                                  MN-major; B = P^T, MN-major)
-// Per CTA (persistent over queries) four warp roles run a pipeline:
-//   warp 0     TMA producer: Q tile per query, K / V rows of each 128-key tile
-//              fetched with tile::gather4 straight into 128B-swizzled smem;
-//   warp 1     MMA issuer (one thread): S^T for tile g, then O^T for tile g-1;
-//   warps 2-5  softmax + epilogue: thread = TMEM lane = key row of the tile.
+// Per CTA (persistent over queries) the warp roles form a pipeline:
+//   warps 0..6   producers: Q tile per query by TMA; the K / V rows of each
+//                128-key tile by cp.async straight into the 128B-swizzled
+//                layout UMMA reads (row gathers through the LSU sustain far
+//                more bandwidth than TMA's four-row gathers);
+//   warp 7       MMA issuer (one thread): S^T of tile g, then O^T of tile g-1;
+//   warps 8..23  four softmax warpgroups, warpgroup w owning heads
+//                [w*H/4, (w+1)*H/4): thread = TMEM lane = key row of the tile.
 // Softmax runs in the exp2 domain with a per-head running maximum that is
 // only raised (and O^T, l rescaled) when a tile exceeds it by more than 2^8,
-// so the cross-thread max reduction happens on the first tile of a query and
-// rarely after. P is rounded to bf16 for the second MMA; accumulation is fp32.
+// so the cross-thread max reduction happens on a query's first tile and
+// rarely after; the per-tile check is one hardware barrier reduction. P is
+// rounded to bf16 for the second MMA; accumulation is fp32.
+//
+// Every mbarrier wait is bounded. Within a softmax warpgroup all four warps
+// take the same sequence of named barriers: a failed wait is folded into the
+// next barrier reduction, after which the whole warpgroup leaves together.
 #include "kernels.cuh"
 #include "tc.cuh"
 
@@ -31,13 +39,15 @@ using namespace tc;
 
 constexpr int D = 128;       // head dim handled by this kernel
 constexpr int TILE = 128;    // kept keys per MMA tile (the M dimension)
+constexpr int NWG = 4;       // softmax warpgroups
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 template <int HP, int NPW>
 struct Cfg {
   static constexpr int NS = HP <= 32 ? 3 : 2;       // K/V pipeline stages
-  static constexpr int HH = HP / 2;                 // heads per softmax warpgroup
-  static constexpr int NWARPS = NPW + 1 + 8;        // producers, MMA issuer, 2 softmax warpgroups
+  static constexpr int HH = HP / NWG;               // heads per softmax warpgroup
+  static constexpr int NSW = 4 * NWG;               // softmax warps
+  static constexpr int NWARPS = NPW + 1 + NSW;
   static constexpr int KV_BYTES = TILE * D * 2;     // one K or V tile: 32 KB
   static constexpr int Q_BYTES = HP * D * 2;        // one query's heads
   static constexpr int P_ROW = HP * 2;              // bytes of one P^T row (<= 128)
@@ -54,7 +64,7 @@ struct Cfg {
 struct Bars {
   uint64_t kfull[3], kempty[3], vfull[3], vempty[3];
   uint64_t qfull[2], qempty[2], sfull[2], sempty[2], pfull[2], pempty[2], ofull[2], oempty[2];
-  uint64_t done, group[2];
+  uint64_t done;
 };
 
 // Bounded wait that also gives up as soon as another role has reported a
@@ -69,26 +79,32 @@ HSA_DEV bool wait_bar(uint64_t* bar, uint32_t parity, bool& dead) {
   dead = true;
   return false;
 }
-
-// Warp-collective form: lane 0 polls, the outcome is broadcast, so every
-// lane of the warp takes the same branch afterwards.
+// Warp form for the producers: lane 0 polls, the outcome is broadcast.
 HSA_DEV bool wait_warp(uint64_t* bar, uint32_t parity, bool& dead) {
   bool ok = false;
   if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, dead);
   ok = __shfl_sync(kFull, ok ? 1 : 0, 0) != 0;
-  __syncwarp();
   dead = !ok;
   return ok;
 }
+// Warp form for the softmax warps: every lane polls, the result is the
+// warp-wide AND (so warp-collective tcgen05 loads stay converged).
+HSA_DEV bool wait_all(uint64_t* bar, uint32_t parity, bool dead) {
+  bool d = dead;
+  const bool ok = wait_bar(bar, parity, d);
+  return __all_sync(kFull, ok);
+}
 
-// Barrier over the four softmax warps on an mbarrier (count 4), bounded like
-// every other wait; `phase` counts the barrier's completed phases.
-HSA_DEV bool group_sync(uint64_t* bar, uint32_t& phase, bool& dead) {
-  __syncwarp();
-  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
-  const bool ok = wait_warp(bar, phase & 1, dead);
-  ++phase;
-  return ok;
+// Named barrier `id` over one softmax warpgroup (128 threads).
+HSA_DEV void wg_sync(int id) { asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory"); }
+HSA_DEV bool wg_or(int id, bool v) {
+  uint32_t out;
+  asm volatile(
+      "{\n .reg .pred a, b;\n setp.ne.u32 a, %2, 0;\n bar.red.or.pred b, %1, 128, a;\n selp.u32 %0, 1, 0, b;\n}"
+      : "=r"(out)
+      : "r"(id), "r"(uint32_t(v))
+      : "memory");
+  return out != 0;
 }
 
 HSA_DEV float redux_max(float v) {
@@ -97,9 +113,8 @@ HSA_DEV float redux_max(float v) {
   return r;
 }
 
-// Sum of v[0..N) over the 32 lanes of a warp by halving exchanges; returns
-// the number of distinct heads each lane ends with (NL) in v[0..NL), lane l
-// holding heads l*NL .. l*NL+NL-1 when N >= 32, else head l / (32/N).
+// Sum of v[0..N) over the 32 lanes of a warp by halving exchanges. Lane l
+// ends with the sums of heads transpose_head<N>(l, e), e < max(N/32, 1).
 template <int N>
 HSA_DEV void warp_transpose_sum(float (&v)[N]) {
   const int lane = threadIdx.x & 31;
@@ -123,52 +138,33 @@ HSA_DEV void warp_transpose_sum(float (&v)[N]) {
     }
   }
 }
-// Head index of value i after warp_transpose_sum<N> in lane `lane`.
 template <int N>
 HSA_DEV int transpose_head(int lane, int i) {
   if (N >= 32) return i + (N / 32) * lane;
-  // n halves log2(N) times using lane bits 4, 3, ... ; the remaining low
-  // lane bits only duplicate.
+  // the halvings consume lane bits 4, 3, ...; the remaining low bits duplicate
   constexpr int shift = (N == 16) ? 1 : (N == 8) ? 2 : (N == 4) ? 3 : (N == 2) ? 4 : 5;
   return lane >> shift;
 }
 
-// HH consecutive TMEM columns of this warp's 32 lanes into v (HH = 8, 16 or 32).
-template <int HH>
-HSA_DEV void tmem_ld_cols(uint32_t taddr, float (&v)[HH]) {
-  if constexpr (HH == 8) {
-    uint32_t r[8];
-    tmem_ld8(taddr, r);
-    tmem_wait_ld();
+// N consecutive 32-bit TMEM columns of this warp's 32 lanes (N = 4, 8, 16).
+template <int N>
+HSA_DEV void tmem_ld_cols(uint32_t taddr, float (&v)[N]) {
+  uint32_t r[N];
+  if constexpr (N == 4) tmem_ld4(taddr, r);
+  else if constexpr (N == 8) tmem_ld8(taddr, r);
+  else tmem_ld16(taddr, r);
+  tmem_wait_ld();
 #pragma unroll
-    for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(r[e]);
-  } else {
-#pragma unroll
-    for (int c0 = 0; c0 < HH; c0 += 16) {
-      uint32_t r[16];
-      tmem_ld16(taddr + c0, r);
-      tmem_wait_ld();
-#pragma unroll
-      for (int e = 0; e < 16; ++e) v[c0 + e] = __uint_as_float(r[e]);
-    }
-  }
+  for (int e = 0; e < N; ++e) v[e] = __uint_as_float(r[e]);
 }
-template <int HH>
-HSA_DEV void tmem_st_cols(uint32_t taddr, const float (&v)[HH]) {
-  if constexpr (HH == 8) {
-    uint32_t r[8];
+template <int N>
+HSA_DEV void tmem_st_cols(uint32_t taddr, const float (&v)[N]) {
+  uint32_t r[N];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) r[e] = __float_as_uint(v[e]);
-    tmem_st8(taddr, r);
-  } else {
-#pragma unroll
-    for (int c0 = 0; c0 < HH; c0 += 16) {
-      uint32_t r[16];
-#pragma unroll
-      for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(v[c0 + e]);
-      tmem_st16(taddr + c0, r);
-    }
-  }
+  for (int e = 0; e < N; ++e) r[e] = __float_as_uint(v[e]);
+  if constexpr (N == 4) tmem_st4(taddr, r);
+  else if constexpr (N == 8) tmem_st8(taddr, r);
+  else tmem_st16(taddr, r);
   tmem_wait_st();
 }
 
@@ -186,7 +182,6 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
   __shared__ float red[4][HP];
   __shared__ float mh[HP];
   __shared__ float lsum[HP];
-  __shared__ int vote[2][2][4];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -195,11 +190,10 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
       mbar_init(&bars.vfull[s], NPW * 32); mbar_init(&bars.vempty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&bars.qfull[b], 1); mbar_init(&bars.qempty[b], 1 + 8);
-      mbar_init(&bars.sfull[b], 1); mbar_init(&bars.sempty[b], 8);
-      mbar_init(&bars.pfull[b], 8); mbar_init(&bars.pempty[b], 1);
-      mbar_init(&bars.ofull[b], 1); mbar_init(&bars.oempty[b], 8);
-      mbar_init(&bars.group[b], 4);
+      mbar_init(&bars.qfull[b], 1); mbar_init(&bars.qempty[b], 1 + C::NSW);
+      mbar_init(&bars.sfull[b], 1); mbar_init(&bars.sempty[b], C::NSW);
+      mbar_init(&bars.pfull[b], C::NSW); mbar_init(&bars.pempty[b], 1);
+      mbar_init(&bars.ofull[b], 1); mbar_init(&bars.oempty[b], C::NSW);
     }
     mbar_init(&bars.done, 1);
     fence_barrier_init();
@@ -214,7 +208,7 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
   if (warp < NPW) {
     // ------------------------------------------------------------ producers
     // Producer thread p copies the (row, 16-byte chunk) pairs p, p + 32*NPW, ...
-    // of each K and V tile with cp.async into the 128B-swizzled layout UMMA reads.
+    // of each K and V tile with cp.async into the 128B-swizzled layout.
     constexpr int PT = NPW * 32, PER = (TILE * 16 + PT - 1) / PT;
     const int p = threadIdx.x;
     if (p == 0) prefetch_tmap(&qmap);
@@ -255,27 +249,27 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
       for (int i = 0; i < nt && !dead; ++i, ++g) {
         const int s = g % C::NS;
         const uint32_t ph = (g / C::NS) & 1;
-        int64_t src[PER];
+        int jr[PER];
         uint32_t dst[PER];
 #pragma unroll
         for (int u = 0; u < PER; ++u) {
           const int e = p + u * PT, r = (e >> 4) & (TILE - 1), c = e & 15;
           const int pos = i * TILE + r;
           const int j = (e < TILE * 16 && pos < k) ? __ldg(row + pos) : -1;
-          src[u] = int64_t((j >= 0 && j < Lk) ? j : 0) * D + c * 8;
+          jr[u] = ((j >= 0 && j < Lk) ? j : 0) * (D / 8) + c;   // 16-byte units
           dst[u] = (c >> 3) * (TILE * 128) + swz_offset(r, c & 7, 128);
         }
         if (!wait_warp(&bars.kempty[s], ph ^ 1, dead)) break;
         const uint32_t kt = smem_u32(sm + C::OFF_K + s * C::KV_BYTES);
 #pragma unroll
         for (int u = 0; u < PER; ++u)
-          if (p + u * PT < TILE * 16) cp_async16(kt + dst[u], K + src[u]);
+          if (p + u * PT < TILE * 16) cp_async16(kt + dst[u], reinterpret_cast<const uint4*>(K) + jr[u]);
         cp_async_arrive(&bars.kfull[s]);
         if (!wait_warp(&bars.vempty[s], ph ^ 1, dead)) break;
         const uint32_t vt = smem_u32(sm + C::OFF_V + s * C::KV_BYTES);
 #pragma unroll
         for (int u = 0; u < PER; ++u)
-          if (p + u * PT < TILE * 16) cp_async16(vt + dst[u], V + src[u]);
+          if (p + u * PT < TILE * 16) cp_async16(vt + dst[u], reinterpret_cast<const uint4*>(V) + jr[u]);
         cp_async_arrive(&bars.vfull[s]);
       }
     }
@@ -297,14 +291,13 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
         if (!wait_bar(&bars.vfull[s], (t.g / C::NS) & 1, dead)) return;
         if (t.first && !wait_bar(&bars.oempty[t.ob], ((t.oq >> 1) & 1) ^ 1, dead)) return;
         tc_fence_after();
-        const uint32_t vbase = smem_u32(sm + C::OFF_V + s * C::KV_BYTES);
-        const uint32_t pbase = smem_u32(sm + C::OFF_P + pb * C::P_BYTES);
+        const uint64_t a0 = smem_desc(smem_u32(sm + C::OFF_V + s * C::KV_BYTES), TILE * 128, 1024, kSw128);
+        const uint64_t b0 = smem_desc(smem_u32(sm + C::OFF_P + pb * C::P_BYTES), 16384, 8 * C::P_ROW, C::P_SWZ);
+        const uint32_t d = tmem + 2 * HP + t.ob * HP;
 #pragma unroll
-        for (int ks = 0; ks < TILE / 16; ++ks) {
-          const uint64_t a = smem_desc(vbase + ks * 2048, TILE * 128, 1024, kSw128);
-          const uint64_t b = smem_desc(pbase + ks * 16 * C::P_ROW, 16384, 8 * C::P_ROW, C::P_SWZ);
-          mma_bf16(tmem + 2 * HP + t.ob * HP, a, b, id_o, (t.first && ks == 0) ? 0u : 1u);
-        }
+        for (int ks = 0; ks < TILE / 16; ++ks)
+          mma_bf16(d, a0 + uint64_t((ks * 2048) >> 4), b0 + uint64_t((ks * 16 * C::P_ROW) >> 4), id_o,
+                   (t.first && ks == 0) ? 0u : 1u);
         mma_commit(&bars.vempty[s]);
         mma_commit(&bars.pempty[pb]);
         if (t.last) mma_commit(&bars.ofull[t.ob]);
@@ -315,19 +308,17 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
         const int nt = qinfo[qb];
         if (nt == 0) { mbar_arrive(&bars.qempty[qb]); continue; }
         const uint32_t ob = oq & 1;
-        const uint32_t qbase = smem_u32(sm + C::OFF_Q + qb * C::Q_BYTES);
+        const uint64_t qd0 = smem_desc(smem_u32(sm + C::OFF_Q + qb * C::Q_BYTES), 16, 1024, kSw128);
         for (int i = 0; i < nt && !dead; ++i, ++g) {
           const int s = g % C::NS, sb = g & 1;
           if (!wait_bar(&bars.kfull[s], (g / C::NS) & 1, dead)) break;
           if (!wait_bar(&bars.sempty[sb], ((g >> 1) & 1) ^ 1, dead)) break;
           tc_fence_after();
-          const uint32_t kbase = smem_u32(sm + C::OFF_K + s * C::KV_BYTES);
+          const uint64_t kd0 = smem_desc(smem_u32(sm + C::OFF_K + s * C::KV_BYTES), 16, 1024, kSw128);
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint64_t a = smem_desc(kbase + (ks / 4) * TILE * 128 + (ks % 4) * 32, 16, 1024, kSw128);
-            const uint64_t b = smem_desc(qbase + (ks / 4) * HP * 128 + (ks % 4) * 32, 16, 1024, kSw128);
-            mma_bf16(tmem + sb * HP, a, b, id_s, ks > 0 ? 1u : 0u);
-          }
+          for (int ks = 0; ks < D / 16; ++ks)
+            mma_bf16(tmem + sb * HP, kd0 + uint64_t(((ks / 4) * TILE * 128 + (ks % 4) * 32) >> 4),
+                     qd0 + uint64_t(((ks / 4) * HP * 128 + (ks % 4) * 32) >> 4), id_s, ks > 0 ? 1u : 0u);
           mma_commit(&bars.kempty[s]);
           mma_commit(&bars.sfull[sb]);
           if (i == nt - 1) mma_commit(&bars.qempty[qb]);
@@ -344,65 +335,64 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax / epilogue
-    // Two warpgroups; warpgroup wg owns heads [wg*HH, wg*HH + HH) of every tile.
-    const int sw = warp - NPW - 1, wg = sw >> 2, wq = sw & 3;
+    const int sw = warp - NPW - 1, wg = sw >> 2;
+    const int bar_id = 1 + wg;
     const int quad = warp & 3;              // TMEM lane quadrant this warp may access
+    const int wq = quad;                    // slot of this warp in the warpgroup's scratch rows
     const int r = quad * 32 + lane;         // key row of the tile / dim row of O^T
     const int h0 = wg * HH;                 // first head of this warpgroup
     const uint32_t lane_addr = uint32_t(quad * 32) << 16;
-    uint64_t* gbar = &bars.group[wg];
-    uint32_t g = 0, qn = 0, oq = 0, gph = 0;
-    for (int q = blockIdx.x; q < Lq && !dead; q += gridDim.x, ++qn) {
+    uint32_t g = 0, qn = 0, oq = 0;
+    for (int q = blockIdx.x; q < Lq; q += gridDim.x, ++qn) {
       const int qb = qn & 1;
-      if (!wait_warp(&bars.qfull[qb], (qn >> 1) & 1, dead)) break;
+      const bool okq = wait_all(&bars.qfull[qb], (qn >> 1) & 1, dead);
+      if (wg_or(bar_id, !okq || dead)) { dead = true; break; }
       const int nt = qinfo[qb];
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.qempty[qb]);
       uint16_t* orow = O + int64_t(q) * H * D;
       if (nt == 0) {
-        for (int h = h0; h < h0 + HH && h < H; ++h) orow[h * D + r] = 0;
+#pragma unroll
+        for (int h = 0; h < HH; ++h)
+          if (h0 + h < H) orow[(h0 + h) * D + r] = 0;
         continue;
       }
       const uint32_t ob = oq & 1;
       const int32_t* irow = idx + int64_t(q) * k;
-      float lp[HH];
+      float lp[HH], m[HH];
 #pragma unroll
-      for (int h = 0; h < HH; ++h) lp[h] = 0.f;
-      for (int i = 0; i < nt && !dead; ++i, ++g) {
+      for (int h = 0; h < HH; ++h) { lp[h] = 0.f; m[h] = -INFINITY; }
+      bool quit = false;
+      for (int i = 0; i < nt; ++i, ++g) {
         const int sb = g & 1;
         const int pos = i * TILE + r;
         const int j = pos < k ? __ldg(irow + pos) : -1;
         const bool valid = j >= 0 && j < Lk;
-        if (!wait_warp(&bars.sfull[sb], (g >> 1) & 1, dead)) break;
-        tc_fence_after();
+        const bool oks = wait_all(&bars.sfull[sb], (g >> 1) & 1, dead);
         float x[HH];
-        tmem_ld_cols<HH>(tmem + lane_addr + sb * HP + h0, x);
+        if (oks) {
+          tc_fence_after();
+          tmem_ld_cols<HH>(tmem + lane_addr + sb * HP + h0, x);
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.sempty[sb]);
+        bool mine = false;
 #pragma unroll
-        for (int h = 0; h < HH; ++h) x[h] = (valid && h0 + h < H) ? x[h] * scale_log2 : -INFINITY;
-
-        // Raise the running maxima only on the first tile, or when some
-        // score exceeds its head's maximum by more than the threshold.
-        bool need_max = (i == 0);
-        if (!need_max) {
-          bool mine = false;
-#pragma unroll
-          for (int h = 0; h < HH; ++h) mine |= x[h] > mh[h0 + h] + kRescaleThreshold;
-          const bool any = __any_sync(kFull, mine);
-          const uint32_t vb = gph & 1;
-          if (lane == 0) vote[vb][wg][wq] = any;
-          if (!group_sync(gbar, gph, dead)) break;
-          need_max = vote[vb][wg][0] | vote[vb][wg][1] | vote[vb][wg][2] | vote[vb][wg][3];
+        for (int h = 0; h < HH; ++h) {
+          x[h] = (oks && valid && h0 + h < H) ? x[h] * scale_log2 : -INFINITY;
+          mine |= x[h] > m[h] + kRescaleThreshold;
         }
-        if (need_max) {
+        dead = dead || !oks;
+        if (wg_or(bar_id, i == 0 || mine || dead)) {
+          if (wg_or(bar_id, dead)) { quit = true; break; }
+          // raise the running maxima of this warpgroup's heads to cover the tile
 #pragma unroll
           for (int h = 0; h < HH; ++h) {
             const float wm = redux_max(x[h]);
             if (lane == (h & 31)) red[wq][h0 + h] = wm;
           }
-          if (!group_sync(gbar, gph, dead)) break;
+          wg_sync(bar_id);
           if (r < HH) {
             const int hh = h0 + r;
             const float tm = fmaxf(fmaxf(red[0][hh], red[1][hh]), fmaxf(red[2][hh], red[3][hh]));
@@ -410,52 +400,64 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
             red[0][hh] = old;  // the previous maximum, for the rescale factors
             mh[hh] = fmaxf(old, tm);
           }
-          if (!group_sync(gbar, gph, dead)) break;
-          if (i > 0) {
-            // rescale l and this warpgroup's O^T columns by 2^(old - new);
-            // the previous tile's PV must have landed first.
-            const uint32_t pg = g - 1;
-            if (!wait_warp(&bars.pempty[pg & 1], (pg >> 1) & 1, dead)) break;
-            tc_fence_after();
-            float ov[HH];
-            const uint32_t ta = tmem + lane_addr + 2 * HP + ob * HP + h0;
-            tmem_ld_cols<HH>(ta, ov);
+          wg_sync(bar_id);
 #pragma unroll
-            for (int h = 0; h < HH; ++h) {
-              const float o = red[0][h0 + h], n = mh[h0 + h];
-              const float a = (o == -INFINITY || n == -INFINITY) ? (o == n ? 1.f : 0.f) : exp2f(o - n);
-              lp[h] *= a;
-              ov[h] *= a;
+          for (int h = 0; h < HH; ++h) m[h] = mh[h0 + h];
+          if (i > 0) {
+            // rescale l and this warpgroup's O^T columns by 2^(old - new); the
+            // previous tile's PV must have landed first
+            const uint32_t pg = g - 1;
+            const bool okp = wait_all(&bars.pempty[pg & 1], (pg >> 1) & 1, dead);
+            dead = dead || !okp;
+            if (okp) {
+              tc_fence_after();
+              float ov[HH];
+              const uint32_t ta = tmem + lane_addr + 2 * HP + ob * HP + h0;
+              tmem_ld_cols<HH>(ta, ov);
+#pragma unroll
+              for (int h = 0; h < HH; ++h) {
+                const float o = red[0][h0 + h], n = m[h];
+                const float a = (o == -INFINITY || n == -INFINITY) ? (o == n ? 1.f : 0.f) : ex2(o - n);
+                lp[h] *= a;
+                ov[h] *= a;
+              }
+              tmem_st_cols<HH>(ta, ov);
             }
-            tmem_st_cols<HH>(ta, ov);
-            // red[0] holds the old maxima until every thread has read them
-            if (!group_sync(gbar, gph, dead)) break;
           }
+          wg_sync(bar_id);  // red[0] holds the old maxima until everyone has read them
         }
         // probabilities, partial row sums, this warpgroup's part of the P^T row
         const int pb = g & 1;
-        if (!wait_warp(&bars.pempty[pb], ((g >> 1) & 1) ^ 1, dead)) break;
-        uint8_t* prow = sm + C::OFF_P + pb * C::P_BYTES;
+        const bool okw = wait_all(&bars.pempty[pb], ((g >> 1) & 1) ^ 1, dead);
+        dead = dead || !okw;
+        uint32_t w[(HH + 1) / 2];
 #pragma unroll
-        for (int c = 0; c < HH / 8; ++c) {
-          uint32_t w[4];
+        for (int e = 0; e < HH / 2; ++e) {
+          // a head with no finite maximum yet has only -inf scores: p = 0
+          const float n0 = m[2 * e] == -INFINITY ? INFINITY : m[2 * e];
+          const float n1 = m[2 * e + 1] == -INFINITY ? INFINITY : m[2 * e + 1];
+          const float p0 = ex2(x[2 * e] - n0), p1 = ex2(x[2 * e + 1] - n1);
+          lp[2 * e] += p0;
+          lp[2 * e + 1] += p1;
+          w[e] = pack_bf16x2(p0, p1);
+        }
+        if (okw) {
+          uint8_t* prow = sm + C::OFF_P + pb * C::P_BYTES;
+          if constexpr (HH >= 8) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int a0 = c * 8 + 2 * e;
-            const float p0 = x[a0] == -INFINITY ? 0.f : exp2f(x[a0] - mh[h0 + a0]);
-            const float p1 = x[a0 + 1] == -INFINITY ? 0.f : exp2f(x[a0 + 1] - mh[h0 + a0 + 1]);
-            lp[a0] += p0;
-            lp[a0 + 1] += p1;
-            w[e] = pack_bf16x2(p0, p1);
+            for (int c = 0; c < HH / 8; ++c)
+              *reinterpret_cast<uint4*>(prow + swz_offset(r, h0 / 8 + c, C::P_ROW)) =
+                  make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+          } else {
+            *reinterpret_cast<uint2*>(prow + swz_offset(r, h0 / 8, C::P_ROW) + (h0 % 8) * 2) = make_uint2(w[0], w[1]);
           }
-          *reinterpret_cast<uint4*>(prow + swz_offset(r, h0 / 8 + c, C::P_ROW)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.pfull[pb]);
       }
-      if (dead) break;
+      if (quit) break;
       // ---- epilogue: row sums, normalise O^T, write O[q][h][r] for this warpgroup's heads
       warp_transpose_sum<HH>(lp);
       constexpr int NL = HH >= 32 ? HH / 32 : 1;
@@ -463,25 +465,27 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
 #pragma unroll
         for (int e = 0; e < NL; ++e) red[wq][h0 + transpose_head<HH>(lane, e)] = lp[e];
       }
-      if (!group_sync(gbar, gph, dead)) break;
+      wg_sync(bar_id);
       if (r < HH) lsum[h0 + r] = red[0][h0 + r] + red[1][h0 + r] + red[2][h0 + r] + red[3][h0 + r];
-      if (!group_sync(gbar, gph, dead)) break;
-      if (!wait_warp(&bars.ofull[ob], (oq >> 1) & 1, dead)) break;
-      tc_fence_after();
-      float ov[HH];
-      tmem_ld_cols<HH>(tmem + lane_addr + 2 * HP + ob * HP + h0, ov);
+      wg_sync(bar_id);
+      const bool oko = wait_all(&bars.ofull[ob], (oq >> 1) & 1, dead);
+      if (oko) {
+        tc_fence_after();
+        float ov[HH];
+        tmem_ld_cols<HH>(tmem + lane_addr + 2 * HP + ob * HP + h0, ov);
 #pragma unroll
-      for (int h = 0; h < HH; ++h) {
-        if (h0 + h < H) {
-          const float l = lsum[h0 + h];
-          orow[(h0 + h) * D + r] = uint16_t(f32_to_bf16_rn(l > 0.f ? ov[h] / l : 0.f));
+        for (int h = 0; h < HH; ++h) {
+          if (h0 + h < H) {
+            const float l = lsum[h0 + h];
+            orow[(h0 + h) * D + r] = uint16_t(f32_to_bf16_rn(l > 0.f ? ov[h] / l : 0.f));
+          }
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.oempty[ob]);
-      // lsum / red are reused by the next query only after the warpgroup is done
-      if (!group_sync(gbar, gph, dead)) break;
+      // also keeps red / lsum untouched until the whole warpgroup is done
+      if (wg_or(bar_id, dead || !oko)) { dead = true; break; }
       ++oq;
     }
   }
@@ -493,8 +497,8 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
   }
 }
 
-// 7 producer warps + 1 MMA warp + 8 softmax warps = 16 warps, 4 per SM
-// sub-partition, which leaves 128 registers per thread.
+// 7 producer warps + 1 MMA warp + 16 softmax warps = 24 warps (6 per SM
+// sub-partition, 80 registers per thread).
 constexpr int kProducerWarps = 7;
 
 template <int HP>
