@@ -359,9 +359,13 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
       }
       const uint32_t ob = oq & 1;
       const int32_t* irow = idx + int64_t(q) * k;
+      // m: running maximum per head (log2 units), or 0 while the head has
+      // seen no valid key (its scores so far are all -inf, so 2^(x - 0) = 0);
+      // `complete`: every real head of this warpgroup has a finite maximum.
       float lp[HH], m[HH];
 #pragma unroll
-      for (int h = 0; h < HH; ++h) { lp[h] = 0.f; m[h] = -INFINITY; }
+      for (int h = 0; h < HH; ++h) { lp[h] = 0.f; m[h] = 0.f; }
+      bool complete = false;
       bool quit = false;
       for (int i = 0; i < nt; ++i, ++g) {
         const int sb = g & 1;
@@ -378,11 +382,13 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.sempty[sb]);
         bool mine = false;
+        const bool live = oks && valid;
 #pragma unroll
         for (int h = 0; h < HH; ++h) {
-          x[h] = (oks && valid && h0 + h < H) ? x[h] * scale_log2 : -INFINITY;
-          mine |= x[h] > m[h] + kRescaleThreshold;
+          x[h] = (live && h0 + h < H) ? x[h] * scale_log2 : -INFINITY;
+          mine |= x[h] - m[h] > kRescaleThreshold;
         }
+        mine |= !complete;
         dead = dead || !oks;
         if (wg_or(bar_id, i == 0 || mine || dead)) {
           if (wg_or(bar_id, dead)) { quit = true; break; }
@@ -401,11 +407,17 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
             mh[hh] = fmaxf(old, tm);
           }
           wg_sync(bar_id);
+          bool all = true;
 #pragma unroll
-          for (int h = 0; h < HH; ++h) m[h] = mh[h0 + h];
+          for (int h = 0; h < HH; ++h) {
+            const float n = mh[h0 + h];
+            m[h] = n == -INFINITY ? 0.f : n;
+            all = all && (n != -INFINITY || h0 + h >= H);
+          }
+          complete = all;
           if (i > 0) {
-            // rescale l and this warpgroup's O^T columns by 2^(old - new); the
-            // previous tile's PV must have landed first
+            // rescale l and this warpgroup's O^T columns; the previous
+            // tile's PV must have landed first
             const uint32_t pg = g - 1;
             const bool okp = wait_all(&bars.pempty[pg & 1], (pg >> 1) & 1, dead);
             dead = dead || !okp;
@@ -416,8 +428,9 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
               tmem_ld_cols<HH>(ta, ov);
 #pragma unroll
               for (int h = 0; h < HH; ++h) {
-                const float o = red[0][h0 + h], n = m[h];
-                const float a = (o == -INFINITY || n == -INFINITY) ? (o == n ? 1.f : 0.f) : ex2(o - n);
+                // o = -inf: nothing accumulated yet (factor 0); n = -inf: no valid key yet
+                const float o = red[0][h0 + h], n = mh[h0 + h];
+                const float a = n == -INFINITY ? 1.f : ex2(o - n);
                 lp[h] *= a;
                 ov[h] *= a;
               }
@@ -433,13 +446,10 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
         uint32_t w[(HH + 1) / 2];
 #pragma unroll
         for (int e = 0; e < HH / 2; ++e) {
-          // a head with no finite maximum yet has only -inf scores: p = 0
-          const float n0 = m[2 * e] == -INFINITY ? INFINITY : m[2 * e];
-          const float n1 = m[2 * e + 1] == -INFINITY ? INFINITY : m[2 * e + 1];
-          const float p0 = ex2(x[2 * e] - n0), p1 = ex2(x[2 * e + 1] - n1);
+          const float p0 = ex2(x[2 * e] - m[2 * e]), p1 = ex2(x[2 * e + 1] - m[2 * e + 1]);
           lp[2 * e] += p0;
           lp[2 * e + 1] += p1;
-          w[e] = pack_bf16x2(p0, p1);
+          w[e] = cvt_bf16x2(p0, p1);
         }
         if (okw) {
           uint8_t* prow = sm + C::OFF_P + pb * C::P_BYTES;

@@ -23,6 +23,12 @@ HSA_DEV uint32_t f32_to_bf16_rn(float f) {
 HSA_DEV uint32_t pack_bf16x2(float lo, float hi) {
   return f32_to_bf16_rn(lo) | (f32_to_bf16_rn(hi) << 16);
 }
+// Same rounding (nearest, ties to even) with the hardware convert.
+HSA_DEV uint32_t cvt_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
 
 // Order-preserving unsigned key of an fp32 score: larger score -> larger key.
 // -0 is folded onto +0 so that the two compare equal, as floats do.
