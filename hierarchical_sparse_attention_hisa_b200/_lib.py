@@ -19,7 +19,7 @@ HSA_OK, HSA_ERR_ARG, HSA_ERR_WORKSPACE, HSA_ERR_CUDA, HSA_ERR_TIMEOUT, HSA_ERR_D
 EXPORTS = (
     "hsa_status_string", "hsa_index_workspace_size", "hsa_block_sums", "hsa_select_blocks",
     "hsa_select_tokens", "hsa_index", "hsa_sparse_attn", "hsa_decode_workspace_size",
-    "hsa_decode_step", "hsa_kernel_launches",
+    "hsa_decode_step", "hsa_kernel_launches", "hsa_decode_step_noalloc",
 )
 
 
@@ -62,6 +62,7 @@ def load():
     L.hsa_sparse_attn.argtypes = [PP, I64, I64, P, P, P, P, P, P]
     L.hsa_decode_workspace_size.argtypes = [PP, I32, I64, ctypes.POINTER(SZ)]
     L.hsa_decode_step.argtypes = [PP, I32, I64, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
+    L.hsa_decode_step_noalloc.argtypes = [PP, I32, I64, P, P, P, P, P, P, P, P, P, P, P, P, P]
     L.hsa_kernel_launches.argtypes, L.hsa_kernel_launches.restype = [], ctypes.c_uint64
     for name in EXPORTS:
         if name not in ("hsa_status_string", "hsa_kernel_launches"):
@@ -153,3 +154,12 @@ def hsa_decode_step(p, batch, capacity, ctx_len, k_idx_cache, K_cache, V_cache, 
         _p(V_cache), _p(ksum_cache), _p(q_idx_new), _p(k_idx_new), _p(Q_new), _p(K_new),
         _p(V_new), _p(O), _p(indices_out), _p(workspace),
         workspace.numel() * workspace.element_size(), _s(stream)))
+
+
+def hsa_decode_step_noalloc(p, batch, capacity, ctx_len, k_idx_cache, K_cache, V_cache, ksum_cache,
+                            q_idx_new, k_idx_new, Q_new, K_new, V_new, O, indices_out, stream=None):
+    """hsa_decode_step with its scratch in the library's static device array."""
+    _check("hsa_decode_step_noalloc", load().hsa_decode_step_noalloc(
+        ctypes.byref(p), batch, capacity, _p(ctx_len), _p(k_idx_cache), _p(K_cache),
+        _p(V_cache), _p(ksum_cache), _p(q_idx_new), _p(k_idx_new), _p(Q_new), _p(K_new),
+        _p(V_new), _p(O), _p(indices_out), _s(stream)))

@@ -158,6 +158,35 @@ HSA_API int hsa_decode_step(const hsa_params* p, int32_t batch, int64_t capacity
                     hsa_bf16* O, int32_t* indices_out, void* workspace, size_t workspace_bytes,
                     cudaStream_t stream);
 
+/* Bytes of the library's static scratch array used by
+ * hsa_decode_step_noalloc (one array per GPU, held from module load until
+ * the process exits). */
+#define HSA_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/* hsa_decode_step without a workspace argument, for callers that cannot
+ * allocate device memory at the point where they decode: code running inside
+ * a framework that owns every allocation (a plugin's enqueue, an embedded
+ * runtime), or a latency-critical serving loop that may not call cudaMalloc
+ * after start-up. The pages describe no such interface; it exists only for
+ * these callers.
+ * Arguments, caches, results and errors are those of hsa_decode_step. The
+ * scratch that hsa_decode_step takes as `workspace` lives instead in a
+ * static device array of HSA_NOALLOC_SCRATCH_BYTES inside the library; a
+ * step needing more (hsa_decode_workspace_size) returns HSA_ERR_WORKSPACE
+ * and launches nothing. Nothing is allocated or freed by this call.
+ * The first call on a device looks up that device's copy of the array
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before capturing the stream into a CUDA graph. Every call on a device
+ * shares the one array and leaves its contents behind: two calls whose work
+ * overlaps on the GPU (different streams without ordering) race on it. */
+HSA_API int hsa_decode_step_noalloc(const hsa_params* p, int32_t batch, int64_t capacity,
+                                    int32_t* ctx_len, hsa_bf16* k_idx_cache, hsa_bf16* K_cache,
+                                    hsa_bf16* V_cache, float* ksum_cache,
+                                    const hsa_bf16* q_idx_new, const hsa_bf16* k_idx_new,
+                                    const hsa_bf16* Q_new, const hsa_bf16* K_new,
+                                    const hsa_bf16* V_new, hsa_bf16* O, int32_t* indices_out,
+                                    cudaStream_t stream);
+
 /* Number of kernels this library has launched in the calling process (all
  * devices, all streams) since it was loaded. A diagnostic counter for
  * benchmarks and tests; it is not synchronised with the GPU. */
