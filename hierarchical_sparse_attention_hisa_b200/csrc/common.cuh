@@ -82,100 +82,267 @@ HSA_DEV int block_exclusive_scan(int v, int* s_tmp, int* total) {
   return res;
 }
 
-// CTA-wide selection of the r largest of n keys (1 <= r <= n), ties broken
-// towards the lowest position. MSB-first radix search with 8-bit digits over
-// the 32-bit keys finds the r-th largest key T; every key > T is taken and,
-// of the keys == T, the `take_eq` at the lowest positions.
+// Block-wide exclusive scan in reverse thread order: thread t gets the sum
+// of v over threads t+1 .. NT-1.
+template <int NT>
+HSA_DEV int block_exclusive_scan_rev(int v, int* s_tmp, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;  // inclusive suffix sum within the warp
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_down_sync(kFull, x, o);
+    if (lane + o < 32) x += y;
+  }
+  if (lane == 0) s_tmp[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < NT / 32 ? s_tmp[lane] : 0;
+    int z = w;  // inclusive suffix over warps
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_down_sync(kFull, z, o);
+      if (lane + o < 32) z += y;
+    }
+    if (lane < NT / 32) s_tmp[lane] = z - w;
+    if (lane == 0) s_tmp[NT / 32] = z;
+  }
+  __syncthreads();
+  int res = s_tmp[warp] + x - v;
+  *total = s_tmp[NT / 32];
+  __syncthreads();
+  return res;
+}
+
+// CTA-wide selection of the r largest of n keys (1 <= r <= n, keys in
+// shared memory), ties broken towards the lowest position.
+// threshold(): the r-th largest key T is found by histogramming the keys
+// relative to their minimum in 2048 bins over the [min, max] range, then
+// narrowing to the bin holding the r-th largest and repeating on that bin
+// (11 bits per round, so at most three rounds; one round when the keys span
+// fewer than 2048 values). take_eq = how many keys equal to T are taken.
+// compact(): emits every selected position in ascending order: all keys > T
+// and the first take_eq keys == T.
 template <int NT>
 struct RadixSelect {
-  uint32_t* hist;   // smem, 256 entries
+  static constexpr int kBins = 2048;
+  static_assert(kBins % NT == 0, "bins per thread");
+  uint32_t* hist;   // smem, kBins entries
   int* scratch;     // smem, NT/32 + 8 ints
 
   HSA_DEV void threshold(const uint32_t* keys, int n, int r, uint32_t* T_out, int* take_eq) {
-    uint32_t prefix = 0, mask = 0;
+    constexpr int NW = NT / 32, BPT = kBins / NT;
+    const int lane = threadIdx.x & 31;
+    volatile int* s = scratch + NW + 2;  // [0]: min, [1]: max, [2]: bin, [3]: above
+    uint32_t lo = 0xffffffffu, hi = 0u;
+    for (int c = threadIdx.x; c < n; c += NT) { const uint32_t u = keys[c]; lo = min(lo, u); hi = max(hi, u); }
+    lo = __reduce_min_sync(kFull, lo);
+    hi = __reduce_max_sync(kFull, hi);
+    if (threadIdx.x == 0) { s[0] = int(0xffffffffu); s[1] = 0; }
+    __syncthreads();
+    if (lane == 0) { atomicMin((unsigned*)&s[0], lo); atomicMax((unsigned*)&s[1], hi); }
+    __syncthreads();
+    uint32_t base = uint32_t(s[0]);
+    uint32_t width = uint32_t(s[1]) - base;  // keys of interest lie in [base, base + width]
     int rem = r;
-    volatile int* s_res = scratch + NT / 32 + 2;  // [digit, above]
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int e = threadIdx.x; e < 256; e += NT) hist[e] = 0;
+    for (;;) {
+      const int bits = 32 - __clz(width);    // bits needed for (key - base)
+      const int shift = bits > 11 ? bits - 11 : 0;
+      for (int e = threadIdx.x; e < kBins; e += NT) hist[e] = 0;
       __syncthreads();
-      for (int c = threadIdx.x; c < n; c += NT) {
-        uint32_t u = keys[c];
-        if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
+      const int per = ((n + NT - 1) / NT);
+      for (int it = 0; it < per; ++it) {
+        const int c = it * NT + threadIdx.x;
+        const uint32_t u = c < n ? keys[c] : 0u;
+        const bool in = c < n && u - base <= width;
+        const uint32_t bin = in ? (u - base) >> shift : 0xffffffffu;
+        const unsigned same = __match_any_sync(kFull, bin);
+        if (in && lane == __ffs(same) - 1) atomicAdd(&hist[bin], __popc(same));
       }
       __syncthreads();
-      if (threadIdx.x < 32) {
-        const int lane = threadIdx.x;
-        uint32_t c8[8], tot = 0;
+      // bins above each thread's BPT bins, via a scan over threads in reverse
+      uint32_t cnt[BPT], tot = 0;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) { c8[e] = hist[lane * 8 + e]; tot += c8[e]; }
-        uint32_t incl = tot;  // sum over lanes >= lane
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          uint32_t y = __shfl_down_sync(kFull, incl, o);
-          if (lane + o < 32) incl += y;
-        }
-        const uint32_t above = incl - tot;
-        if (above < uint32_t(rem) && uint32_t(rem) <= incl) {
-          uint32_t a = above;
-          for (int e = 7; e >= 0; --e) {
-            if (a + c8[e] >= uint32_t(rem)) { s_res[0] = lane * 8 + e; s_res[1] = int(a); break; }
-            a += c8[e];
-          }
+      for (int e = 0; e < BPT; ++e) { cnt[e] = hist[threadIdx.x * BPT + e]; tot += cnt[e]; }
+      int total;
+      // exclusive scan in reversed thread order = counts of all bins above mine
+      int above = block_exclusive_scan_rev<NT>(int(tot), scratch, &total);
+      if (uint32_t(above) < uint32_t(rem) && uint32_t(rem) <= uint32_t(above) + tot) {
+        uint32_t a = uint32_t(above);
+        for (int e = BPT - 1; e >= 0; --e) {
+          if (a + cnt[e] >= uint32_t(rem)) { s[2] = threadIdx.x * BPT + e; s[3] = int(a); break; }
+          a += cnt[e];
         }
       }
       __syncthreads();
-      const uint32_t digit = uint32_t(s_res[0]);
-      rem -= s_res[1];
-      prefix |= digit << shift;
-      mask |= 255u << shift;
+      const uint32_t bin = uint32_t(s[2]);
+      rem -= s[3];
+      base += bin << shift;
+      const uint32_t span = shift ? ((1u << shift) - 1u) : 0u;
+      width = min(span, uint32_t(s[1]) - base);
       __syncthreads();
+      if (shift == 0) break;
     }
-    *T_out = prefix;
+    *T_out = base;
     *take_eq = rem;
   }
 
-  // Writes the positions of the selected keys, ascending, via emit(rank, pos).
-  // Warps own contiguous position ranges; lanes interleave inside them.
+  // Emits (rank, pos) for every selected position, ascending. Warps own
+  // contiguous position ranges; lanes interleave inside them. A position's
+  // rank is (#keys > T before it) + min(#keys == T before it, take_eq).
   template <class Emit>
   HSA_DEV void compact(const uint32_t* keys, int n, uint32_t T, int take_eq, Emit emit) {
     constexpr int NW = NT / 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int per = ((n + NW * 32 - 1) / (NW * 32)) * 32;
     const int lo = warp * per, hi = min(n, lo + per);
-    int neq = 0;
+    int ngt = 0, neq = 0;
     for (int c0 = lo; c0 < hi; c0 += 32) {
       const int c = c0 + lane;
-      neq += __popc(__ballot_sync(kFull, c < hi && keys[c] == T));
+      const uint32_t u = c < hi ? keys[c] : 0u;
+      ngt += __popc(__ballot_sync(kFull, c < hi && u > T));
+      neq += __popc(__ballot_sync(kFull, c < hi && u == T));
     }
     int tot;
-    int eq_before = block_exclusive_scan<NT>(lane == 0 ? neq : 0, scratch, &tot);
-    eq_before = __shfl_sync(kFull, eq_before, 0);
-    int nsel = 0, eqs = eq_before;
+    // one scan over the packed pair (counts < 2^15 per CTA for n <= 16384)
+    const int packed = block_exclusive_scan<NT>(lane == 0 ? (ngt << 16) | neq : 0, scratch, &tot);
+    const int pk = __shfl_sync(kFull, packed, 0);
+    int gt_before = pk >> 16, eq_before = pk & 0xffff;
     for (int c0 = lo; c0 < hi; c0 += 32) {
       const int c = c0 + lane;
       const uint32_t u = c < hi ? keys[c] : 0u;
+      const unsigned bgt = __ballot_sync(kFull, c < hi && u > T);
       const unsigned beq = __ballot_sync(kFull, c < hi && u == T);
-      const int my_eq_rank = eqs + __popc(beq & ((1u << lane) - 1u));
-      const bool sel = c < hi && (u > T || (u == T && my_eq_rank < take_eq));
-      nsel += __popc(__ballot_sync(kFull, sel));
-      eqs += __popc(beq);
-    }
-    int sel_before = block_exclusive_scan<NT>(lane == 0 ? nsel : 0, scratch, &tot);
-    sel_before = __shfl_sync(kFull, sel_before, 0);
-    eqs = eq_before;
-    int out = sel_before;
-    for (int c0 = lo; c0 < hi; c0 += 32) {
-      const int c = c0 + lane;
-      const uint32_t u = c < hi ? keys[c] : 0u;
-      const unsigned beq = __ballot_sync(kFull, c < hi && u == T);
-      const int my_eq_rank = eqs + __popc(beq & ((1u << lane) - 1u));
-      const bool sel = c < hi && (u > T || (u == T && my_eq_rank < take_eq));
-      const unsigned bs = __ballot_sync(kFull, sel);
-      if (sel) emit(out + __popc(bs & ((1u << lane) - 1u)), c);
-      out += __popc(bs);
-      eqs += __popc(beq);
+      const unsigned below = (1u << lane) - 1u;
+      const int g_me = gt_before + __popc(bgt & below);
+      const int e_me = eq_before + __popc(beq & below);
+      if (c < hi && (u > T || (u == T && e_me < take_eq))) emit(g_me + min(e_me, take_eq), c);
+      gt_before += __popc(bgt);
+      eq_before += __popc(beq);
     }
   }
 };
+
+// Selection of the r largest of n keys (1 <= r <= n) held in registers:
+// thread t holds positions [t*KPT, t*KPT + KPT), positions >= n are ignored.
+// Ties go to the lowest position. threshold() histograms the keys relative
+// to their minimum in 2048 bins over [min, max] and narrows to the bin that
+// holds the r-th largest key, 11 bits per round; compact() emits every
+// selected position in ascending order with its rank (#keys > T before it +
+// min(#keys == T before it, take_eq)).
+template <int NT, int KPT>
+struct RegSelect {
+  static constexpr int kBins = 2048;
+  static_assert(kBins % NT == 0, "bins per thread");
+  uint32_t* hist;   // smem, kBins entries
+  int* scratch;     // smem, NT/32 + 8 ints
+
+  HSA_DEV void threshold(const uint32_t (&key)[KPT], int n, int r, uint32_t* T_out, int* take_eq) {
+    constexpr int NW = NT / 32, BPT = kBins / NT;
+    const int lane = threadIdx.x & 31;
+    volatile int* s = scratch + NW + 2;  // [0] min, [1] max, [2] bin, [3] above
+    const int p0 = threadIdx.x * KPT;
+    uint32_t lo = 0xffffffffu, hi = 0u;
+#pragma unroll
+    for (int j = 0; j < KPT; ++j)
+      if (p0 + j < n) { lo = min(lo, key[j]); hi = max(hi, key[j]); }
+    lo = __reduce_min_sync(kFull, lo);
+    hi = __reduce_max_sync(kFull, hi);
+    if (threadIdx.x == 0) { s[0] = int(0xffffffffu); s[1] = 0; }
+    __syncthreads();
+    if (lane == 0) { atomicMin((unsigned*)&s[0], lo); atomicMax((unsigned*)&s[1], hi); }
+    __syncthreads();
+    const uint32_t kmax = uint32_t(s[1]);
+    uint32_t base = uint32_t(s[0]);
+    uint32_t width = kmax - base;
+    int rem = r;
+    for (;;) {
+      const int bits = 32 - __clz(width);
+      const int shift = bits > 11 ? bits - 11 : 0;
+#pragma unroll
+      for (int e = 0; e < BPT; ++e) hist[threadIdx.x * BPT + e] = 0;
+      __syncthreads();
+#pragma unroll
+      for (int j = 0; j < KPT; ++j) {
+        const uint32_t d = key[j] - base;
+        if (p0 + j < n && d <= width) atomicAdd(&hist[d >> shift], 1u);
+      }
+      __syncthreads();
+      uint32_t cnt[BPT], tot = 0;
+#pragma unroll
+      for (int e = 0; e < BPT; ++e) { cnt[e] = hist[threadIdx.x * BPT + e]; tot += cnt[e]; }
+      int total;
+      const int above = block_exclusive_scan_rev<NT>(int(tot), scratch, &total);
+      if (uint32_t(above) < uint32_t(rem) && uint32_t(rem) <= uint32_t(above) + tot) {
+        uint32_t a = uint32_t(above);
+#pragma unroll
+        for (int e = BPT - 1; e >= 0; --e) {
+          if (a + cnt[e] >= uint32_t(rem)) { s[2] = threadIdx.x * BPT + e; s[3] = int(a); break; }
+          a += cnt[e];
+        }
+      }
+      __syncthreads();
+      const uint32_t bin = uint32_t(s[2]);
+      rem -= s[3];
+      const bool whole = hist[bin] == uint32_t(rem);  // every key of the bin is taken
+      base += bin << shift;
+      width = min(shift ? (1u << shift) - 1u : 0u, kmax - base);
+      __syncthreads();
+      if (whole && base > 0u) {
+        // select every key >= base: threshold just below the bin, no ties taken
+        *T_out = base - 1u;
+        *take_eq = 0;
+        return;
+      }
+      if (shift == 0) break;
+    }
+    *T_out = base;
+    *take_eq = rem;
+  }
+
+  template <class Emit>
+  HSA_DEV void compact(const uint32_t (&key)[KPT], int n, uint32_t T, int take_eq, Emit emit) {
+    const int p0 = threadIdx.x * KPT;
+    int ngt = 0, neq = 0;
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+      ngt += (p0 + j < n && key[j] > T);
+      neq += (p0 + j < n && key[j] == T);
+    }
+    int tot;
+    // counts stay below 2^15 per CTA (n <= 16384), so one packed scan serves both
+    const int packed = block_exclusive_scan<NT>((ngt << 16) | neq, scratch, &tot);
+    int gt = packed >> 16, eq = packed & 0xffff;
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+      if (p0 + j >= n) break;
+      if (key[j] > T) {
+        emit(gt + min(eq, take_eq), p0 + j);
+        ++gt;
+      } else if (key[j] == T) {
+        if (eq < take_eq) emit(gt + eq, p0 + j);
+        ++eq;
+      }
+    }
+  }
+};
+
+// Loads keys [p0, p0 + KPT) of row (p0 = threadIdx.x * KPT), 16 bytes at a
+// time where the row is 16-byte aligned and complete.
+template <int KPT>
+HSA_DEV void load_keys(const uint32_t* __restrict__ row, int n, uint32_t (&key)[KPT]) {
+  const int p0 = threadIdx.x * KPT;
+  if constexpr (KPT % 4 == 0) {
+    if (p0 + KPT <= n && (reinterpret_cast<uintptr_t>(row) & 15u) == 0) {
+#pragma unroll
+      for (int v = 0; v < KPT / 4; ++v) {
+        const uint4 q = __ldg(reinterpret_cast<const uint4*>(row + p0) + v);
+        key[4 * v] = q.x; key[4 * v + 1] = q.y; key[4 * v + 2] = q.z; key[4 * v + 3] = q.w;
+      }
+      return;
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) key[j] = p0 + j < n ? __ldg(row + p0 + j) : 0u;
+}
 
 }  // namespace hsa

@@ -87,7 +87,7 @@ __global__ void __launch_bounds__(256) select_blocks_kernel(RowMap rm, const uin
                                                             int32_t* __restrict__ blocks) {
   constexpr int NT = 256;
   extern __shared__ __align__(16) uint32_t smem_u32[];
-  __shared__ uint32_t hist[256];
+  __shared__ uint32_t hist[RadixSelect<NT>::kBins];
   __shared__ int scratch[NT / 32 + 8];
   __shared__ float qs[D];
   const int64_t i = blockIdx.x;
@@ -165,7 +165,7 @@ __global__ void __launch_bounds__(256) select_tokens_kernel(RowMap rm, const uin
                                                             int m, int k, int32_t* __restrict__ indices) {
   constexpr int NT = 256;
   extern __shared__ __align__(16) uint32_t smem_u32[];
-  __shared__ uint32_t hist[256];
+  __shared__ uint32_t hist[RadixSelect<NT>::kBins];
   __shared__ int scratch[NT / 32 + 8];
   __shared__ float qs[D];
   __shared__ int blk[256];

@@ -13,6 +13,7 @@ namespace hsa {
 namespace {
 
 constexpr int NT = 256;
+constexpr int NT_TOPK = 512;  // top-k rows hold up to m*B keys: 16 per thread at 8192
 
 // Kept-block list of one row: count of valid entries and candidate count
 // (tokens j <= t of the kept blocks). Returns false when the list does not
@@ -28,10 +29,10 @@ HSA_DEV bool row_candidates(const int32_t* blk, int m, int64_t t, int B, int* nb
   return true;
 }
 
+template <int KPT>
 __global__ void __launch_bounds__(NT) topm_from_keys_kernel(RowMap rm, const uint32_t* __restrict__ bkeys,
                                                            int64_t ld, int B, int m, int32_t* __restrict__ blocks) {
-  extern __shared__ __align__(16) uint32_t keys[];
-  __shared__ uint32_t hist[256];
+  __shared__ uint32_t hist[RegSelect<NT, KPT>::kBins];
   __shared__ int scratch[NT / 32 + 8];
   const int64_t i = blockIdx.x;
   int32_t* out = blocks + i * m;
@@ -46,15 +47,14 @@ __global__ void __launch_bounds__(NT) topm_from_keys_kernel(RowMap rm, const uin
     return;
   }
   const int n = int(nb - 2);  // candidates: blocks 1 .. nb-2
-  const uint32_t* row = bkeys + i * ld + 1;
-  for (int c = threadIdx.x; c < n; c += NT) keys[c] = row[c];
-  __syncthreads();
-  RadixSelect<NT> rs{hist, scratch};
+  uint32_t key[KPT];
+  load_keys<KPT>(bkeys + i * ld + 1, n, key);
+  RegSelect<NT, KPT> rs{hist, scratch};
   uint32_t T;
   int take_eq;
-  rs.threshold(keys, n, m - 2, &T, &take_eq);
+  rs.threshold(key, n, m - 2, &T, &take_eq);
   if (threadIdx.x == 0) { out[0] = 0; out[m - 1] = int32_t(nb - 1); }
-  rs.compact(keys, n, T, take_eq, [&](int rank, int c) { out[1 + rank] = c + 1; });
+  rs.compact(key, n, T, take_eq, [&](int rank, int c) { out[1 + rank] = c + 1; });
 }
 
 // Pairs of the rows [r0, r0 + ROWS) that need token scores, binned by block.
@@ -132,11 +132,12 @@ __global__ void __launch_bounds__(1024) pair_scan_kernel(int nbins, const int* _
   if (threadIdx.x == 0) *ntiles = carry_tiles;
 }
 
-__global__ void __launch_bounds__(NT) topk_from_keys_kernel(RowMap rm, const int32_t* __restrict__ blocks,
-                                                           const uint32_t* __restrict__ tkeys, int B, int m,
-                                                           int k, int32_t* __restrict__ indices) {
-  extern __shared__ __align__(16) uint32_t keys[];
-  __shared__ uint32_t hist[256];
+template <int KPT>
+__global__ void __launch_bounds__(NT_TOPK) topk_from_keys_kernel(RowMap rm, const int32_t* __restrict__ blocks,
+                                                                const uint32_t* __restrict__ tkeys, int B, int m,
+                                                                int k, int32_t* __restrict__ indices) {
+  constexpr int NT = NT_TOPK;
+  __shared__ uint32_t hist[RegSelect<NT, KPT>::kBins];
   __shared__ int scratch[NT / 32 + 8];
   __shared__ int blk[256];
   __shared__ int s_info[3];
@@ -157,33 +158,51 @@ __global__ void __launch_bounds__(NT) topk_from_keys_kernel(RowMap rm, const int
     return;
   }
   const int n = s_info[2];
-  auto tok = [&](int c) -> int32_t { return int32_t(int64_t(blk[c / B]) * B + c % B); };
+  const bool pow2 = (B & (B - 1)) == 0;
+  const int lb = 31 - __clz(B);
+  auto tok = [&](int c) -> int32_t {
+    return pow2 ? (blk[c >> lb] << lb) + (c & (B - 1)) : int32_t(int64_t(blk[c / B]) * B + c % B);
+  };
   if (n <= k) {
     for (int s = threadIdx.x; s < k; s += NT) out[s] = s < n ? tok(s) : -1;
     return;
   }
-  const uint32_t* row = tkeys + i * int64_t(m) * B;
-  const int n4 = n / 4;
-  for (int c = threadIdx.x; c < n4; c += NT)
-    reinterpret_cast<uint4*>(keys)[c] = __ldg(reinterpret_cast<const uint4*>(row) + c);
-  for (int c = n4 * 4 + threadIdx.x; c < n; c += NT) keys[c] = row[c];
-  __syncthreads();
-  RadixSelect<NT> rs{hist, scratch};
+  uint32_t key[KPT];
+  load_keys<KPT>(tkeys + i * int64_t(m) * B, n, key);
+  RegSelect<NT, KPT> rs{hist, scratch};
   uint32_t T;
   int take_eq;
-  rs.threshold(keys, n, k, &T, &take_eq);
-  rs.compact(keys, n, T, take_eq, [&](int rank, int c) { out[rank] = tok(c); });
+  rs.threshold(key, n, k, &T, &take_eq);
+  rs.compact(key, n, T, take_eq, [&](int rank, int c) { out[rank] = tok(c); });
 }
 
 }  // namespace
+
+// Keys per thread for up to n keys over NT threads: 1, 2, 4, ..., 64.
+static int keys_per_thread(int64_t n) {
+  int kpt = 1;
+  while (int64_t(kpt) * NT < n) kpt *= 2;
+  return kpt;
+}
+
+#define HSA_KPT_DISPATCH(kpt, CALL) \
+  switch (kpt) {                    \
+    case 1: CALL(1); break;         \
+    case 2: CALL(2); break;         \
+    case 4: CALL(4); break;         \
+    case 8: CALL(8); break;         \
+    case 16: CALL(16); break;       \
+    case 32: CALL(32); break;       \
+    default: CALL(64); break;       \
+  }
 
 void launch_topm_from_keys(RowMap rm, int64_t rows, const uint32_t* bkeys, int64_t ld, int B, int m,
                            int64_t max_cand, int32_t* blocks, cudaStream_t s) {
   if (rows == 0) return;
   count_launches(1);
-  const size_t smem = size_t(max_cand > 0 ? max_cand : 1) * 4;
-  cudaFuncSetAttribute(topm_from_keys_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  topm_from_keys_kernel<<<unsigned(rows), NT, smem, s>>>(rm, bkeys, ld, B, m, blocks);
+#define HSA_TOPM(K) topm_from_keys_kernel<K><<<unsigned(rows), NT, 0, s>>>(rm, bkeys, ld, B, m, blocks)
+  HSA_KPT_DISPATCH(keys_per_thread(max_cand), HSA_TOPM)
+#undef HSA_TOPM
 }
 
 void launch_pair_lists(RowMap rm, int64_t rows, const int32_t* blocks, int B, int m, int k, int nbins,
@@ -205,9 +224,11 @@ void launch_topk_from_keys(RowMap rm, int64_t rows, const int32_t* blocks, const
                            int m, int k, int32_t* indices, cudaStream_t s) {
   if (rows == 0) return;
   count_launches(1);
-  const size_t smem = size_t(m) * B * 4;
-  cudaFuncSetAttribute(topk_from_keys_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  topk_from_keys_kernel<<<unsigned(rows), NT, smem, s>>>(rm, blocks, tkeys, B, m, k, indices);
+#define HSA_TOPK(K) topk_from_keys_kernel<K><<<unsigned(rows), NT_TOPK, 0, s>>>(rm, blocks, tkeys, B, m, k, indices)
+  int kpt = 1;
+  while (int64_t(kpt) * NT_TOPK < int64_t(m) * B) kpt *= 2;
+  HSA_KPT_DISPATCH(kpt, HSA_TOPK)
+#undef HSA_TOPK
 }
 
 }  // namespace hsa
