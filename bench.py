@@ -253,7 +253,7 @@ def bench_decode(args, world, device):
     import hierarchical_sparse_attention_hisa_b200 as hsa
 
     w = DECODE
-    steps = max(1, min(args.decode_steps, w.decode_steps))
+    steps = max(2, min(args.decode_steps, w.decode_steps))
     warm = min(args.warmup, 8)
     cap = w.decode_ctx + warm + steps + w.B
     cap = (cap + w.B - 1) // w.B * w.B
@@ -271,22 +271,46 @@ def bench_decode(args, world, device):
     stream = torch.cuda.current_stream()
 
     def step(s):
+        # launched on the current stream: the capture stream inside the graph
         hsa.hsa_decode_step(p, w.batch, cap, ctx, kc, Kc, Vc, ksum, new["q_idx_new"][s],
                             new["k_idx_new"][s], new["Q_new"][s], new["K_new"][s], new["V_new"][s],
-                            O, idx, ws, stream)
+                            O, idx, ws, None)
 
     for s in range(warm):
         step(s)
     torch.cuda.synchronize()
+    # direct launches of a few steps, for reference
+    n_direct = min(8, steps // 2)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for s in range(warm, warm + n_direct):
+        step(s)
+    b.record()
+    torch.cuda.synchronize()
+    ms_direct = a.elapsed_time(b) / max(1, n_direct)
+    warm += n_direct
+    steps -= n_direct
+    # the timed steps are captured once into a CUDA graph (each step's own
+    # input rows baked in) and replayed, as a serving loop would
+    graph = torch.cuda.CUDAGraph()
+    launches0 = hsa.kernel_launches()
+    with torch.cuda.graph(graph):
+        for s in range(warm, warm + steps):
+            step(s)
+    launches = hsa.kernel_launches() - launches0
+    torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
+    stream = torch.cuda.current_stream()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
-    for s in range(warm, warm + steps):
-        step(s)
+    graph.replay()
     b.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(a.elapsed_time(b) / steps, world, device)
+    del graph
+    # every captured step ran: each sequence grew by one token per step
+    assert int(ctx.min().item()) == int(ctx.max().item()) == w.decode_ctx + warm + steps, "decode graph did not run"
     hbm, _, _, src = peaks()
     # algorithmic bytes per query: block sums read + kept blocks' index keys +
     # kept K/V rows + Q and O rows
@@ -295,7 +319,9 @@ def bench_decode(args, world, device):
     gbs = per_q * w.batch / (ms / 1e3) / 1e9
     return {"metric": "decode queries/s at 128K", "value": w.batch * world / (ms / 1e3),
             "unit": "queries/s", "ms_per_step": ms, "steps": steps, "batch": w.batch,
-            "ctx": w.decode_ctx, "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm,
+            "ctx": w.decode_ctx, "timing": "CUDA graph of the timed steps, CUDA events",
+            "ms_per_step_direct_launch": ms_direct, "gpu_launches": int(launches),
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm,
                                               "unit": "GB/s", "frac": gbs / hbm,
                                               "peak_source": src,
                                               "bytes_per_query": per_q}}

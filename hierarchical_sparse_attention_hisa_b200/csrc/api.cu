@@ -1,5 +1,6 @@
 // C ABI of libhsa.so (declared in include/hsa.h): host-side argument checks,
 // workspace layout and kernel launches. No allocation, no synchronisation.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -279,14 +280,47 @@ int hsa_sparse_attn(const hsa_params* p, int64_t Lq, int64_t Lk, const hsa_bf16*
   return launch_status();
 }
 
+}  // extern "C"
+
+namespace {
+
+// Workspace of a decode step (256-byte aligned regions):
+//   blocks [batch][m] i32, indices [batch][k] i32 (unless the caller takes them),
+//   block-score keys [batch][capacity/B] u32, token-score keys [batch][m*B] u32,
+//   attention parts: O [batch*parts][H][d] f32, maxima and row sums [batch*parts][H] f32.
+struct DecodeWs {
+  size_t blocks, idx, bkeys, tkeys, opart, mpart, lpart, total;
+  int parts;
+};
+DecodeWs decode_ws(const hsa_params* p, int32_t batch, int64_t capacity) {
+  DecodeWs w{};
+  const int tiles = (p->k + 127) / 128;
+  // enough parts per query to give every SM work at small batch
+  w.parts = batch > 0 ? std::max(1, std::min(tiles, 128 / std::max(1, int(batch)))) : 1;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { const size_t at = o; o += align_up(bytes > 0 ? bytes : 1); return at; };
+  w.blocks = take(size_t(batch) * p->m * 4);
+  w.idx = take(size_t(batch) * p->k * 4);
+  w.bkeys = take(size_t(batch) * (capacity / p->B) * 4);
+  w.tkeys = take(size_t(batch) * p->m * p->B * 4);
+  w.opart = take(size_t(batch) * w.parts * p->H * p->d * 4);
+  w.mpart = take(size_t(batch) * w.parts * p->H * 4);
+  w.lpart = take(size_t(batch) * w.parts * p->H * 4);
+  w.total = o;
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
 int hsa_decode_workspace_size(const hsa_params* p, int32_t batch, int64_t capacity,
                               size_t* bytes) {
   if (!bytes) return HSA_ERR_ARG;
   if (int e = check_index_params(p)) return e;
   if (int e = check_attn_params(p)) return e;
   if (batch < 0 || capacity < p->B || capacity % p->B) return HSA_ERR_ARG;
-  *bytes = align_up(size_t(batch) * p->m * sizeof(int32_t)) +
-           align_up(size_t(batch) * p->k * sizeof(int32_t));
+  *bytes = decode_ws(p, batch, capacity).total;
   return HSA_OK;
 }
 
@@ -300,27 +334,47 @@ int hsa_decode_step(const hsa_params* p, int32_t batch, int64_t capacity, int32_
   if (int e = hsa_decode_workspace_size(p, batch, capacity, &need)) return e;
   if (capacity / p->B > kMaxCandidates || capacity > (int64_t(1) << 31) - 1) return HSA_ERR_ARG;
   if (batch == 0) return HSA_OK;
-  const void* ptrs[] = {ctx_len, k_idx_cache, K_cache, V_cache, ksum_cache, q_idx_new,
+  const void* ptrs[] = {k_idx_cache, K_cache, V_cache, ksum_cache, q_idx_new,
                         k_idx_new, Q_new, K_new, V_new, O};
   for (const void* q : ptrs)
-    if (!aligned16(q) && q != ctx_len) return HSA_ERR_ARG;
+    if (!aligned16(q)) return HSA_ERR_ARG;
   if (!ctx_len || (reinterpret_cast<uintptr_t>(ctx_len) & 3u)) return HSA_ERR_ARG;
   if (indices_out && !aligned16(indices_out)) return HSA_ERR_ARG;
   if (!aligned16(workspace) || workspace_bytes < need) return HSA_ERR_WORKSPACE;
   if (int e = check_device()) return e;
+  const DecodeWs w = decode_ws(p, batch, capacity);
   char* ws = static_cast<char*>(workspace);
-  int32_t* blocks = reinterpret_cast<int32_t*>(ws);
-  int32_t* idx = indices_out ? indices_out
-                             : reinterpret_cast<int32_t*>(ws + align_up(size_t(batch) * p->m * 4));
+  int32_t* blocks = reinterpret_cast<int32_t*>(ws + w.blocks);
+  int32_t* idx = indices_out ? indices_out : reinterpret_cast<int32_t*>(ws + w.idx);
+  uint32_t* bkeys = reinterpret_cast<uint32_t*>(ws + w.bkeys);
+  uint32_t* tkeys = reinterpret_cast<uint32_t*>(ws + w.tkeys);
+  const int64_t nbc = capacity / p->B;
+  hsa::RowMap rm{batch, capacity, ctx_len, capacity};
+  // 1. append the new token (and the block sum of a block it completes)
   hsa::launch_decode_append(batch, capacity, ctx_len, p->B, p->d_idx, p->d, k_idx_cache, K_cache,
                             V_cache, ksum_cache, k_idx_new, K_new, V_new, stream);
-  hsa::RowMap rm{batch, capacity, ctx_len, capacity};
-  hsa::launch_select_blocks(rm, batch, q_idx_new, ksum_cache, (capacity / p->B) * p->d_idx, p->B,
-                            p->m, p->d_idx, blocks, capacity / p->B, stream);
-  hsa::launch_select_tokens(rm, batch, q_idx_new, k_idx_cache, blocks, p->B, p->m, p->k,
-                            p->d_idx, idx, stream);
-  hsa::launch_sparse_attn_simple(rm, batch, Q_new, K_cache, V_cache, idx, p->k, p->H, p->d,
-                                 softmax_scale(p), O, stream);
+  // 2. block scores against the block-sum cache, top-m with the forced blocks
+  hsa::launch_decode_block_scores(batch, capacity, ctx_len, p->B, p->m, p->d_idx, q_idx_new, ksum_cache,
+                                  bkeys, nbc, stream);
+  hsa::launch_topm_from_keys(rm, batch, bkeys, nbc, p->B, p->m, nbc > 2 ? nbc - 2 : 1, blocks, stream);
+  // 3. token scores inside the kept blocks, top-k
+  hsa::launch_decode_token_scores(batch, capacity, ctx_len, p->B, p->m, p->d_idx, blocks, q_idx_new,
+                                  k_idx_cache, tkeys, stream);
+  hsa::launch_topk_from_keys(rm, batch, blocks, tkeys, p->B, p->m, p->k, idx, stream);
+  // 4. attention over the kept tokens: parts of each query on the tensor cores, then combined
+  if (hsa::tc_attn_supported(p->H, p->d, batch, capacity)) {
+    float* opart = reinterpret_cast<float*>(ws + w.opart);
+    float* mpart = reinterpret_cast<float*>(ws + w.mpart);
+    float* lpart = reinterpret_cast<float*>(ws + w.lpart);
+    if (!hsa::launch_sparse_attn_tc_split(batch, Q_new, K_cache, V_cache, idx, capacity, p->k, p->H,
+                                          softmax_scale(p), w.parts, opart, mpart, lpart, stream))
+      return HSA_ERR_CUDA;
+    hsa::launch_decode_combine(batch, capacity, ctx_len, p->H, p->d, w.parts, opart, mpart, lpart, O, stream);
+  } else {
+    hsa::launch_sparse_attn_simple(rm, batch, Q_new, K_cache, V_cache, idx, p->k, p->H, p->d,
+                                   softmax_scale(p), O, stream);
+  }
+  // 5. the sequences grow by one token
   hsa::launch_decode_advance(batch, capacity, ctx_len, stream);
   return launch_status();
 }

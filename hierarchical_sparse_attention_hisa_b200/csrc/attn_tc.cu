@@ -67,6 +67,26 @@ struct Bars {
   uint64_t done;
 };
 
+}  // namespace
+
+// Work description of one launch. Query q's kept indices are idx[q][0..k);
+// its K/V rows start at row q * kv_stride (0: one K/V shared by all queries).
+// Each query is cut into items_per_query parts of tiles_per_item 128-key
+// tiles; with one part per query the kernel writes normalised O, otherwise
+// every part w = q * items_per_query + s writes its unnormalised O^T, running
+// maximum and row sum for a later combination.
+struct AttnArgs {
+  const int32_t* idx;
+  int Lq, Lk, k, H;
+  float scale_log2;
+  int64_t kv_stride;
+  int items_per_query, tiles_per_item;
+  uint16_t* O;
+  float *Opart, *mpart, *lpart;  // [items][H][D], [items][H], [items][H]
+};
+
+namespace {
+
 // Bounded wait that also gives up as soon as another role has reported a
 // failure, so one lost arrival cannot keep any warp spinning for long.
 HSA_DEV bool wait_bar(uint64_t* bar, uint32_t parity, bool& dead) {
@@ -171,14 +191,19 @@ HSA_DEV void tmem_st_cols(uint32_t taddr, const float (&v)[N]) {
 template <int HP, int NPW>
 __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_kernel(
     const __grid_constant__ CUtensorMap qmap, const uint16_t* __restrict__ K, const uint16_t* __restrict__ V,
-    const int32_t* __restrict__ idx, int Lq, int Lk, int k, int H, float scale_log2, uint16_t* __restrict__ O) {
+    const AttnArgs a) {
   using C = Cfg<HP, NPW>;
+  const int32_t* __restrict__ idx = a.idx;
+  const int Lk = a.Lk, k = a.k, H = a.H;
+  const float scale_log2 = a.scale_log2;
+  const int ipq = a.items_per_query, tpi = a.tiles_per_item;
+  const int n_items = a.Lq * ipq;
   constexpr int HH = C::HH;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ __align__(8) Bars bars;
   __shared__ uint32_t tmem_base;
-  __shared__ int qinfo[2];
+  __shared__ int qinfo[2][2];  // per Q buffer: first tile, tile count
   __shared__ float red[4][HP];
   __shared__ float mh[HP];
   __shared__ float lsum[HP];
@@ -213,8 +238,11 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
     const int p = threadIdx.x;
     if (p == 0) prefetch_tmap(&qmap);
     uint32_t g = 0, qn = 0;
-    for (int q = blockIdx.x; q < Lq && !dead; q += gridDim.x, ++qn) {
+    for (int w = blockIdx.x; w < n_items && !dead; w += gridDim.x, ++qn) {
+      const int q = w / ipq, part = w - q * ipq;
       const int32_t* row = idx + int64_t(q) * k;
+      const uint4* Kq = reinterpret_cast<const uint4*>(K + int64_t(q) * a.kv_stride * D);
+      const uint4* Vq = reinterpret_cast<const uint4*>(V + int64_t(q) * a.kv_stride * D);
       int last = -1;  // tiles = ceil((last valid position + 1) / TILE)
       if ((k & 3) == 0) {
         const int4* row4 = reinterpret_cast<const int4*>(row);
@@ -234,12 +262,14 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
       }
 #pragma unroll
       for (int o = 16; o >= 1; o >>= 1) last = max(last, __shfl_xor_sync(kFull, last, o));
-      const int nt = (last + TILE) / TILE;
+      const int t0 = part * tpi;                                  // this item's tiles
+      const int nt = max(0, min((last + TILE) / TILE, t0 + tpi) - t0);
       const int qb = qn & 1;
       if (warp == 0) {
         if (!wait_warp(&bars.qempty[qb], ((qn >> 1) & 1) ^ 1, dead)) break;
         if (lane == 0) {
-          qinfo[qb] = nt;
+          qinfo[qb][0] = t0;
+          qinfo[qb][1] = nt;
           mbar_arrive_expect_tx(&bars.qfull[qb], C::Q_BYTES);
           uint8_t* qt = sm + C::OFF_Q + qb * C::Q_BYTES;
           tma_load_2d(qt, &qmap, &bars.qfull[qb], 0, q * H);
@@ -254,7 +284,7 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
 #pragma unroll
         for (int u = 0; u < PER; ++u) {
           const int e = p + u * PT, r = (e >> 4) & (TILE - 1), c = e & 15;
-          const int pos = i * TILE + r;
+          const int pos = (t0 + i) * TILE + r;
           const int j = (e < TILE * 16 && pos < k) ? __ldg(row + pos) : -1;
           jr[u] = ((j >= 0 && j < Lk) ? j : 0) * (D / 8) + c;   // 16-byte units
           dst[u] = (c >> 3) * (TILE * 128) + swz_offset(r, c & 7, 128);
@@ -263,13 +293,13 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
         const uint32_t kt = smem_u32(sm + C::OFF_K + s * C::KV_BYTES);
 #pragma unroll
         for (int u = 0; u < PER; ++u)
-          if (p + u * PT < TILE * 16) cp_async16(kt + dst[u], reinterpret_cast<const uint4*>(K) + jr[u]);
+          if (p + u * PT < TILE * 16) cp_async16(kt + dst[u], Kq + jr[u]);
         cp_async_arrive(&bars.kfull[s]);
         if (!wait_warp(&bars.vempty[s], ph ^ 1, dead)) break;
         const uint32_t vt = smem_u32(sm + C::OFF_V + s * C::KV_BYTES);
 #pragma unroll
         for (int u = 0; u < PER; ++u)
-          if (p + u * PT < TILE * 16) cp_async16(vt + dst[u], reinterpret_cast<const uint4*>(V) + jr[u]);
+          if (p + u * PT < TILE * 16) cp_async16(vt + dst[u], Vq + jr[u]);
         cp_async_arrive(&bars.vfull[s]);
       }
     }
@@ -302,10 +332,10 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
         mma_commit(&bars.pempty[pb]);
         if (t.last) mma_commit(&bars.ofull[t.ob]);
       };
-      for (int q = blockIdx.x; q < Lq && !dead; q += gridDim.x, ++qn) {
+      for (int w = blockIdx.x; w < n_items && !dead; w += gridDim.x, ++qn) {
         const int qb = qn & 1;
         if (!wait_bar(&bars.qfull[qb], (qn >> 1) & 1, dead)) break;
-        const int nt = qinfo[qb];
+        const int nt = qinfo[qb][1];
         if (nt == 0) { mbar_arrive(&bars.qempty[qb]); continue; }
         const uint32_t ob = oq & 1;
         const uint64_t qd0 = smem_desc(smem_u32(sm + C::OFF_Q + qb * C::Q_BYTES), 16, 1024, kSw128);
@@ -343,18 +373,24 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
     const int h0 = wg * HH;                 // first head of this warpgroup
     const uint32_t lane_addr = uint32_t(quad * 32) << 16;
     uint32_t g = 0, qn = 0, oq = 0;
-    for (int q = blockIdx.x; q < Lq; q += gridDim.x, ++qn) {
+    for (int w = blockIdx.x; w < n_items; w += gridDim.x, ++qn) {
+      const int q = w / ipq;
       const int qb = qn & 1;
       const bool okq = wait_all(&bars.qfull[qb], (qn >> 1) & 1, dead);
       if (wg_or(bar_id, !okq || dead)) { dead = true; break; }
-      const int nt = qinfo[qb];
+      const int t0 = qinfo[qb][0], nt = qinfo[qb][1];
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.qempty[qb]);
-      uint16_t* orow = O + int64_t(q) * H * D;
+      uint16_t* orow = a.O ? a.O + int64_t(q) * H * D : nullptr;
       if (nt == 0) {
+        if (orow) {
 #pragma unroll
-        for (int h = 0; h < HH; ++h)
-          if (h0 + h < H) orow[(h0 + h) * D + r] = 0;
+          for (int h = 0; h < HH; ++h)
+            if (h0 + h < H) orow[(h0 + h) * D + r] = 0;
+        } else if (r < HH && h0 + r < H) {  // an empty part: no weight in the combination
+          a.mpart[int64_t(w) * H + h0 + r] = -INFINITY;
+          a.lpart[int64_t(w) * H + h0 + r] = 0.f;
+        }
         continue;
       }
       const uint32_t ob = oq & 1;
@@ -369,7 +405,7 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
       bool quit = false;
       for (int i = 0; i < nt; ++i, ++g) {
         const int sb = g & 1;
-        const int pos = i * TILE + r;
+        const int pos = (t0 + i) * TILE + r;
         const int j = pos < k ? __ldg(irow + pos) : -1;
         const bool valid = j >= 0 && j < Lk;
         const bool oks = wait_all(&bars.sfull[sb], (g >> 1) & 1, dead);
@@ -483,11 +519,23 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
         tc_fence_after();
         float ov[HH];
         tmem_ld_cols<HH>(tmem + lane_addr + 2 * HP + ob * HP + h0, ov);
+        if (orow) {
 #pragma unroll
-        for (int h = 0; h < HH; ++h) {
-          if (h0 + h < H) {
-            const float l = lsum[h0 + h];
-            orow[(h0 + h) * D + r] = uint16_t(f32_to_bf16_rn(l > 0.f ? ov[h] / l : 0.f));
+          for (int h = 0; h < HH; ++h) {
+            if (h0 + h < H) {
+              const float l = lsum[h0 + h];
+              orow[(h0 + h) * D + r] = uint16_t(f32_to_bf16_rn(l > 0.f ? ov[h] / l : 0.f));
+            }
+          }
+        } else {
+          // one part of a split query: unnormalised O^T, running maximum, row sum
+          float* op = a.Opart + int64_t(w) * H * D;
+#pragma unroll
+          for (int h = 0; h < HH; ++h)
+            if (h0 + h < H) op[(h0 + h) * D + r] = ov[h];
+          if (r < HH && h0 + r < H) {
+            a.mpart[int64_t(w) * H + h0 + r] = mh[h0 + r];
+            a.lpart[int64_t(w) * H + h0 + r] = lsum[h0 + r];
           }
         }
       }
@@ -512,18 +560,24 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
 constexpr int kProducerWarps = 7;
 
 template <int HP>
-bool launch_hp(const void* Q, const void* K, const void* V, const int32_t* idx, int Lq, int Lk, int k,
-               int H, float scale_log2, void* O, cudaStream_t s) {
+bool launch_hp(const void* Q, const void* K, const void* V, const AttnArgs& a, cudaStream_t s) {
   CUtensorMap qm;
-  if (!make_tmap_2d(&qm, Q, uint64_t(Lq) * H, D, HP)) return false;
+  if (!make_tmap_2d(&qm, Q, uint64_t(a.Lq) * a.H, D, HP)) return false;
   using C = Cfg<HP, kProducerWarps>;
   auto kern = sparse_attn_tc_kernel<HP, kProducerWarps>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
     return false;
-  const int grid = Lq < num_sms() ? Lq : num_sms();
-  kern<<<grid, 32 * C::NWARPS, C::SMEM, s>>>(qm, static_cast<const uint16_t*>(K), static_cast<const uint16_t*>(V),
-                                             idx, Lq, Lk, k, H, scale_log2, static_cast<uint16_t*>(O));
+  const int64_t items = int64_t(a.Lq) * a.items_per_query;
+  const int grid = int(items < num_sms() ? items : num_sms());
+  kern<<<grid, 32 * C::NWARPS, C::SMEM, s>>>(qm, static_cast<const uint16_t*>(K), static_cast<const uint16_t*>(V), a);
   return true;
+}
+
+bool launch_args(const void* Q, const void* K, const void* V, const AttnArgs& a, cudaStream_t s) {
+  count_launches(1);
+  if (a.H <= 16) return launch_hp<16>(Q, K, V, a, s);
+  if (a.H <= 32) return launch_hp<32>(Q, K, V, a, s);
+  return launch_hp<64>(Q, K, V, a, s);
 }
 
 }  // namespace
@@ -538,12 +592,29 @@ bool tc_attn_supported(int H, int d, int64_t Lq, int64_t Lk) {
 bool launch_sparse_attn_tc(int64_t Lq, const void* Q, const void* K, const void* V, const int32_t* idx,
                            int64_t Lk, int k, int H, float scale, void* O, cudaStream_t s) {
   if (Lq == 0) return true;
-  count_launches(1);
-  const float sl2 = scale * 1.4426950408889634f;
-  const int L = int(Lq), LK = int(Lk);
-  if (H <= 16) return launch_hp<16>(Q, K, V, idx, L, LK, k, H, sl2, O, s);
-  if (H <= 32) return launch_hp<32>(Q, K, V, idx, L, LK, k, H, sl2, O, s);
-  return launch_hp<64>(Q, K, V, idx, L, LK, k, H, sl2, O, s);
+  AttnArgs a{};
+  a.idx = idx; a.Lq = int(Lq); a.Lk = int(Lk); a.k = k; a.H = H;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.kv_stride = 0;
+  a.items_per_query = 1;
+  a.tiles_per_item = (k + TILE - 1) / TILE;
+  a.O = static_cast<uint16_t*>(O);
+  return launch_args(Q, K, V, a, s);
+}
+
+bool launch_sparse_attn_tc_split(int batch, const void* Q, const void* Kc, const void* Vc, const int32_t* idx,
+                                 int64_t capacity, int k, int H, float scale, int parts, float* Opart,
+                                 float* mpart, float* lpart, cudaStream_t s) {
+  if (batch == 0) return true;
+  AttnArgs a{};
+  a.idx = idx; a.Lq = batch; a.Lk = int(capacity); a.k = k; a.H = H;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.kv_stride = capacity;
+  a.items_per_query = parts;
+  a.tiles_per_item = ((k + TILE - 1) / TILE + parts - 1) / parts;
+  a.O = nullptr;
+  a.Opart = Opart; a.mpart = mpart; a.lpart = lpart;
+  return launch_args(Q, Kc, Vc, a, s);
 }
 
 }  // namespace hsa

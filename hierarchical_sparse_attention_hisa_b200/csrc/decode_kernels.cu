@@ -35,6 +35,159 @@ __global__ void __launch_bounds__(128) decode_append_kernel(
   }
 }
 
+// Block scores of the new query of sequence b against its complete blocks
+// 1 .. nb-2 (blocks 0 and nb-1 are forced, so never scored): one warp per
+// block row of the fp32 block-sum cache, fp32 products reduced across the
+// warp, written as order-preserving keys bkeys[b][block].
+template <int DI>
+__global__ void __launch_bounds__(256) decode_block_scores_kernel(const int32_t* __restrict__ ctx, int64_t capacity,
+                                                                  int B, int m, int per_cta,
+                                                                  const uint16_t* __restrict__ q_new,
+                                                                  const float* __restrict__ ksum_cache,
+                                                                  uint32_t* __restrict__ bkeys, int64_t ld) {
+  constexpr int VPL = DI / 32;  // fp32 values per lane
+  const int64_t b = blockIdx.x;
+  const int64_t t = ctx[b];
+  if (t < 0 || t >= capacity) return;
+  const int64_t nb = t / B + 1;
+  if (nb <= m) return;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float q[VPL];
+#pragma unroll
+  for (int e = 0; e < VPL; ++e) q[e] = __uint_as_float(uint32_t(q_new[b * DI + lane * VPL + e]) << 16);
+  const int64_t lo = 1 + int64_t(blockIdx.y) * per_cta, hi = min(nb - 1, lo + per_cta);
+  const float* base = ksum_cache + b * (capacity / B) * DI;
+  for (int64_t blk = lo + warp; blk < hi; blk += 8) {
+    const float* row = base + blk * DI + lane * VPL;
+    float acc = 0.f;
+    if constexpr (VPL == 4) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(row));
+      acc = q[0] * v.x;
+      acc = __fmaf_rn(q[1], v.y, acc);
+      acc = __fmaf_rn(q[2], v.z, acc);
+      acc = __fmaf_rn(q[3], v.w, acc);
+    } else {
+      const float2 v = __ldg(reinterpret_cast<const float2*>(row));
+      acc = q[0] * v.x;
+      acc = __fmaf_rn(q[1], v.y, acc);
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
+    if (lane == 0) bkeys[b * ld + blk] = score_key(acc);
+  }
+}
+
+// Token scores of sequence b's new query against the B keys of its kept
+// block in slot s: a half-warp per key row (16-byte loads), written as keys
+// tkeys[b][s][r]. Rows past the query's position are scored too but never
+// read: the selection takes only the first candidate-count entries.
+template <int DI>
+__global__ void __launch_bounds__(128) decode_token_scores_kernel(const int32_t* __restrict__ ctx, int64_t capacity,
+                                                                  int B, int m, const int32_t* __restrict__ blocks,
+                                                                  const uint16_t* __restrict__ q_new,
+                                                                  const uint16_t* __restrict__ k_idx_cache,
+                                                                  uint32_t* __restrict__ tkeys) {
+  constexpr int LPR = DI / 8;          // lanes per row (8 bf16 each)
+  constexpr int RPW = 32 / LPR;        // rows per warp instruction
+  const int64_t b = blockIdx.x;
+  const int s = blockIdx.y;
+  const int64_t t = ctx[b];
+  if (t < 0 || t >= capacity) return;
+  const int blk = blocks[b * m + s];
+  if (blk < 0) return;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int sub = lane % LPR, rsub = lane / LPR;
+  const uint4 qv = __ldg(reinterpret_cast<const uint4*>(q_new + b * DI) + sub);
+  const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+  const uint16_t* kb = k_idx_cache + (b * capacity + int64_t(blk) * B) * DI;
+  uint32_t* out = tkeys + (b * m + s) * int64_t(B);
+  for (int r0 = warp * RPW; r0 < B; r0 += 4 * RPW) {
+    const int r = r0 + rsub;
+    float acc = 0.f;
+    if (r < B) {
+      const uint4 kv = __ldg(reinterpret_cast<const uint4*>(kb + int64_t(r) * DI) + sub);
+      const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc = __fmaf_rn(bf16_lo(qw[e]), bf16_lo(kw[e]), acc);
+        acc = __fmaf_rn(bf16_hi(qw[e]), bf16_hi(kw[e]), acc);
+      }
+    }
+#pragma unroll
+    for (int o = LPR / 2; o >= 1; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
+    if (sub == 0 && r < B) out[r] = score_key(acc);
+  }
+}
+
+// O[b][h][:] from the parts of a split query: with M the largest part
+// maximum, O = sum_p 2^(m_p - M) O_p / sum_p 2^(m_p - M) l_p (log2 units).
+// One CTA per (sequence, head), one thread per output element.
+__global__ void decode_combine_kernel(const int32_t* __restrict__ ctx, int64_t capacity, int H, int D, int parts,
+                                      const float* __restrict__ Opart, const float* __restrict__ mpart,
+                                      const float* __restrict__ lpart, uint16_t* __restrict__ O) {
+  const int64_t b = blockIdx.x / H;
+  const int h = blockIdx.x % H;
+  const int64_t t = ctx[b];
+  float out = 0.f;
+  if (t >= 0 && t < capacity) {
+    float M = -INFINITY;
+    for (int p = 0; p < parts; ++p) {
+      const int64_t w = b * parts + p;
+      if (lpart[w * H + h] > 0.f) M = fmaxf(M, mpart[w * H + h]);
+    }
+    float num = 0.f, den = 0.f;
+    for (int p = 0; p < parts; ++p) {
+      const int64_t w = b * parts + p;
+      const float l = lpart[w * H + h];
+      if (l > 0.f) {
+        const float f = exp2f(mpart[w * H + h] - M);
+        num = __fmaf_rn(f, Opart[(w * H + h) * D + threadIdx.x], num);
+        den = __fmaf_rn(f, l, den);
+      }
+    }
+    out = den > 0.f ? num / den : 0.f;
+  }
+  O[(b * H + h) * D + threadIdx.x] = uint16_t(f32_to_bf16_rn(out));
+}
+
+void launch_decode_block_scores(int batch, int64_t capacity, const int32_t* ctx, int B, int m, int d_idx,
+                                const void* q_new, const float* ksum_cache, uint32_t* bkeys, int64_t ld,
+                                cudaStream_t s) {
+  if (batch == 0) return;
+  const int64_t nbmax = capacity / B;
+  const int per_cta = 128;
+  const dim3 grid((unsigned)batch, (unsigned)((nbmax + per_cta - 1) / per_cta));
+  count_launches(1);
+  if (d_idx == 128)
+    decode_block_scores_kernel<128><<<grid, 256, 0, s>>>(ctx, capacity, B, m, per_cta, (const uint16_t*)q_new,
+                                                         ksum_cache, bkeys, ld);
+  else
+    decode_block_scores_kernel<64><<<grid, 256, 0, s>>>(ctx, capacity, B, m, per_cta, (const uint16_t*)q_new,
+                                                        ksum_cache, bkeys, ld);
+}
+
+void launch_decode_token_scores(int batch, int64_t capacity, const int32_t* ctx, int B, int m, int d_idx,
+                                const int32_t* blocks, const void* q_new, const void* k_idx_cache,
+                                uint32_t* tkeys, cudaStream_t s) {
+  if (batch == 0) return;
+  const dim3 grid((unsigned)batch, (unsigned)m);
+  count_launches(1);
+  if (d_idx == 128)
+    decode_token_scores_kernel<128><<<grid, 128, 0, s>>>(ctx, capacity, B, m, blocks, (const uint16_t*)q_new,
+                                                         (const uint16_t*)k_idx_cache, tkeys);
+  else
+    decode_token_scores_kernel<64><<<grid, 128, 0, s>>>(ctx, capacity, B, m, blocks, (const uint16_t*)q_new,
+                                                        (const uint16_t*)k_idx_cache, tkeys);
+}
+
+void launch_decode_combine(int batch, int64_t capacity, const int32_t* ctx, int H, int d, int parts,
+                           const float* Opart, const float* mpart, const float* lpart, void* O, cudaStream_t s) {
+  if (batch == 0) return;
+  count_launches(1);
+  decode_combine_kernel<<<unsigned(batch * H), d, 0, s>>>(ctx, capacity, H, d, parts, Opart, mpart, lpart,
+                                                         (uint16_t*)O);
+}
+
 __global__ void decode_advance_kernel(int batch, int64_t capacity, int32_t* ctx) {
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b < batch && ctx[b] >= 0 && ctx[b] < capacity) ctx[b] += 1;

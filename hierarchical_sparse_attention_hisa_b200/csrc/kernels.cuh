@@ -50,6 +50,17 @@ void launch_decode_append(int batch, int64_t capacity, const int32_t* ctx, int B
                           void* k_idx_cache, void* K_cache, void* V_cache, float* ksum_cache,
                           const void* k_idx_new, const void* K_new, const void* V_new,
                           cudaStream_t s);
+void launch_decode_block_scores(int batch, int64_t capacity, const int32_t* ctx, int B, int m, int d_idx,
+                                const void* q_new, const float* ksum_cache, uint32_t* bkeys, int64_t ld,
+                                cudaStream_t s);
+void launch_decode_token_scores(int batch, int64_t capacity, const int32_t* ctx, int B, int m, int d_idx,
+                                const int32_t* blocks, const void* q_new, const void* k_idx_cache,
+                                uint32_t* tkeys, cudaStream_t s);
+void launch_decode_combine(int batch, int64_t capacity, const int32_t* ctx, int H, int d, int parts,
+                           const float* Opart, const float* mpart, const float* lpart, void* O, cudaStream_t s);
+bool launch_sparse_attn_tc_split(int batch, const void* Q, const void* Kc, const void* Vc, const int32_t* idx,
+                                 int64_t capacity, int k, int H, float scale, int parts, float* Opart,
+                                 float* mpart, float* lpart, cudaStream_t s);
 void launch_decode_advance(int batch, int64_t capacity, int32_t* ctx, cudaStream_t s);
 
 }  // namespace hsa

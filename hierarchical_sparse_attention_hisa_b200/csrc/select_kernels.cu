@@ -36,6 +36,10 @@ __global__ void __launch_bounds__(NT) topm_from_keys_kernel(RowMap rm, const uin
   __shared__ int scratch[NT / 32 + 8];
   const int64_t i = blockIdx.x;
   int32_t* out = blocks + i * m;
+  if (!rm.valid(i)) {
+    for (int s = threadIdx.x; s < m; s += NT) out[s] = -1;
+    return;
+  }
   const int64_t t = rm.pos(i);
   const int64_t nb = t / B + 1;
   if (nb <= m) {
@@ -132,17 +136,20 @@ __global__ void __launch_bounds__(1024) pair_scan_kernel(int nbins, const int* _
   if (threadIdx.x == 0) *ntiles = carry_tiles;
 }
 
-template <int KPT>
-__global__ void __launch_bounds__(NT_TOPK) topk_from_keys_kernel(RowMap rm, const int32_t* __restrict__ blocks,
-                                                                const uint32_t* __restrict__ tkeys, int B, int m,
-                                                                int k, int32_t* __restrict__ indices) {
-  constexpr int NT = NT_TOPK;
+template <int NT, int KPT>
+__global__ void __launch_bounds__(NT) topk_from_keys_kernel(RowMap rm, const int32_t* __restrict__ blocks,
+                                                           const uint32_t* __restrict__ tkeys, int B, int m,
+                                                           int k, int32_t* __restrict__ indices) {
   __shared__ uint32_t hist[RegSelect<NT, KPT>::kBins];
   __shared__ int scratch[NT / 32 + 8];
   __shared__ int blk[256];
   __shared__ int s_info[3];
   const int64_t i = blockIdx.x;
   int32_t* out = indices + i * int64_t(k);
+  if (!rm.valid(i)) {
+    for (int s = threadIdx.x; s < k; s += NT) out[s] = -1;
+    return;
+  }
   const int64_t t = rm.pos(i);
   for (int s = threadIdx.x; s < m; s += NT) blk[s] = blocks[i * m + s];
   __syncthreads();
@@ -224,11 +231,21 @@ void launch_topk_from_keys(RowMap rm, int64_t rows, const int32_t* blocks, const
                            int m, int k, int32_t* indices, cudaStream_t s) {
   if (rows == 0) return;
   count_launches(1);
-#define HSA_TOPK(K) topk_from_keys_kernel<K><<<unsigned(rows), NT_TOPK, 0, s>>>(rm, blocks, tkeys, B, m, k, indices)
-  int kpt = 1;
-  while (int64_t(kpt) * NT_TOPK < int64_t(m) * B) kpt *= 2;
-  HSA_KPT_DISPATCH(kpt, HSA_TOPK)
+  // few rows (a decode batch): wide CTAs cut each row's latency; many rows:
+  // 512 threads keep several CTAs per SM
+  if (rows < 2 * num_sms()) {
+#define HSA_TOPK(K) topk_from_keys_kernel<1024, K><<<unsigned(rows), 1024, 0, s>>>(rm, blocks, tkeys, B, m, k, indices)
+    int kpt = 1;
+    while (int64_t(kpt) * 1024 < int64_t(m) * B) kpt *= 2;
+    HSA_KPT_DISPATCH(kpt, HSA_TOPK)
 #undef HSA_TOPK
+  } else {
+#define HSA_TOPK(K) topk_from_keys_kernel<NT_TOPK, K><<<unsigned(rows), NT_TOPK, 0, s>>>(rm, blocks, tkeys, B, m, k, indices)
+    int kpt = 1;
+    while (int64_t(kpt) * NT_TOPK < int64_t(m) * B) kpt *= 2;
+    HSA_KPT_DISPATCH(kpt, HSA_TOPK)
+#undef HSA_TOPK
+  }
 }
 
 }  // namespace hsa
