@@ -382,6 +382,40 @@ def bench_reference(args, rank, world):
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+# ---------------------------------------------------------------- profiling cases
+
+def profile_case(name):
+    """Small cases for ncu captures: the last 8192 queries of the 64K workload
+    (inputs larger than L2), run three times untimed and once timed."""
+    import torch
+    import hierarchical_sparse_attention_hisa_b200 as hsa
+    hsa.load()
+    w = PREFILL
+    lq = 8192
+    x = synth.prefill_inputs(w, with_attn=(name == "attn_last8k"))
+    dev = lambda u: dev_bf16(u, "cuda")  # noqa: E731
+    q_idx, k_idx = dev(x["q_idx"][-lq:]), dev(x["k_idx"])
+    p = hsa.params(B=w.B, m=w.m, k=w.k, d_idx=w.d_idx, H=w.H, d=w.d)
+    ws = torch.empty(hsa.hsa_index_workspace_size(p, lq, w.L), dtype=torch.uint8, device="cuda")
+    idx = torch.empty((lq, w.k), dtype=torch.int32, device="cuda")
+    if name == "attn_last8k":
+        Q, K, V = dev(x["Q"][-lq:]), dev(x["K"]), dev(x["V"])
+        O = torch.empty_like(Q)
+        hsa.hsa_index(p, lq, w.L, q_idx, k_idx, idx, ws)
+        run = lambda: hsa.hsa_sparse_attn(p, lq, w.L, Q, K, V, idx, O)  # noqa: E731
+    else:
+        run = lambda: hsa.hsa_index(p, lq, w.L, q_idx, k_idx, idx, ws)  # noqa: E731
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    run()
+    b.record()
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": name, "ms": a.elapsed_time(b)}))
+
+
 # ---------------------------------------------------------------- main
 
 def main():
@@ -394,7 +428,12 @@ def main():
     ap.add_argument("--skip-decode", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", choices=["attn_last8k", "index_last8k"],
+                    help="run one small case for an ncu capture and exit")
     args = ap.parse_args()
+    if args.profile_case:
+        profile_case(args.profile_case)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -237,31 +237,39 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
     constexpr int PT = NPW * 32, PER = (TILE * 16 + PT - 1) / PT;
     const int p = threadIdx.x;
     if (p == 0) prefetch_tmap(&qmap);
+    // The tile count of a query needs its last valid index position: the
+    // row is searched backwards 128 entries at a time, and the last 128
+    // entries of the next query's row are fetched one query ahead, so the
+    // usual case (a valid tail) costs no exposed load latency.
+    const bool vec = (k & 3) == 0 && k >= 128;
+    const int s0 = vec ? k - 128 : 0;  // start of the last 128-entry window
+    auto tail_window = [&](int q) -> int4 {
+      return vec ? __ldg(reinterpret_cast<const int4*>(idx + int64_t(q) * k + s0) + lane) : make_int4(-1, -1, -1, -1);
+    };
+    int4 pre = blockIdx.x < n_items ? tail_window(blockIdx.x / ipq) : make_int4(-1, -1, -1, -1);
     uint32_t g = 0, qn = 0;
     for (int w = blockIdx.x; w < n_items && !dead; w += gridDim.x, ++qn) {
       const int q = w / ipq, part = w - q * ipq;
       const int32_t* row = idx + int64_t(q) * k;
       const uint4* Kq = reinterpret_cast<const uint4*>(K + int64_t(q) * a.kv_stride * D);
       const uint4* Vq = reinterpret_cast<const uint4*>(V + int64_t(q) * a.kv_stride * D);
+      const int4 win = pre;
+      if (w + int(gridDim.x) < n_items) pre = tail_window((w + gridDim.x) / ipq);
       int last = -1;  // tiles = ceil((last valid position + 1) / TILE)
-      if ((k & 3) == 0) {
-        const int4* row4 = reinterpret_cast<const int4*>(row);
-#pragma unroll 4
-        for (int p4 = lane; p4 < k / 4; p4 += 32) {
-          const int4 v = __ldg(row4 + p4);
-          if (v.x >= 0 && v.x < Lk) last = 4 * p4;
-          if (v.y >= 0 && v.y < Lk) last = 4 * p4 + 1;
-          if (v.z >= 0 && v.z < Lk) last = 4 * p4 + 2;
-          if (v.w >= 0 && v.w < Lk) last = 4 * p4 + 3;
-        }
-      } else {
-        for (int pp = lane; pp < k; pp += 32) {
-          const int j = __ldg(row + pp);
-          if (j >= 0 && j < Lk) last = pp;
-        }
+      if (vec) {
+        if (win.x >= 0 && win.x < Lk) last = s0 + 4 * lane;
+        if (win.y >= 0 && win.y < Lk) last = s0 + 4 * lane + 1;
+        if (win.z >= 0 && win.z < Lk) last = s0 + 4 * lane + 2;
+        if (win.w >= 0 && win.w < Lk) last = s0 + 4 * lane + 3;
       }
 #pragma unroll
       for (int o = 16; o >= 1; o >>= 1) last = max(last, __shfl_xor_sync(kFull, last, o));
+      for (int c0 = (vec ? s0 : k) - 32; last < 0 && c0 > -32; c0 -= 32) {  // backwards, 32 at a time
+        const int pp = c0 + lane;
+        const int j = pp >= 0 ? __ldg(row + pp) : -1;
+        const unsigned v = __ballot_sync(kFull, j >= 0 && j < Lk);
+        if (v) last = c0 + 31 - __clz(v);
+      }
       const int t0 = part * tpi;                                  // this item's tiles
       const int nt = max(0, min((last + TILE) / TILE, t0 + tpi) - t0);
       const int qb = qn & 1;
@@ -289,13 +297,15 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
           jr[u] = ((j >= 0 && j < Lk) ? j : 0) * (D / 8) + c;   // 16-byte units
           dst[u] = (c >> 3) * (TILE * 128) + swz_offset(r, c & 7, 128);
         }
-        if (!wait_warp(&bars.kempty[s], ph ^ 1, dead)) break;
+        // with two stages, a K stage is free once S of the tile two back is
+        // done (sfull), a V stage once its PV is done (pempty)
+        if (!wait_warp(C::NS == 2 ? &bars.sfull[s] : &bars.kempty[s], ph ^ 1, dead)) break;
         const uint32_t kt = smem_u32(sm + C::OFF_K + s * C::KV_BYTES);
 #pragma unroll
         for (int u = 0; u < PER; ++u)
           if (p + u * PT < TILE * 16) cp_async16(kt + dst[u], Kq + jr[u]);
         cp_async_arrive(&bars.kfull[s]);
-        if (!wait_warp(&bars.vempty[s], ph ^ 1, dead)) break;
+        if (!wait_warp(C::NS == 2 ? &bars.pempty[s] : &bars.vempty[s], ph ^ 1, dead)) break;
         const uint32_t vt = smem_u32(sm + C::OFF_V + s * C::KV_BYTES);
 #pragma unroll
         for (int u = 0; u < PER; ++u)
@@ -328,7 +338,7 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
         for (int ks = 0; ks < TILE / 16; ++ks)
           mma_bf16(d, a0 + uint64_t((ks * 2048) >> 4), b0 + uint64_t((ks * 16 * C::P_ROW) >> 4), id_o,
                    (t.first && ks == 0) ? 0u : 1u);
-        mma_commit(&bars.vempty[s]);
+        if (C::NS != 2) mma_commit(&bars.vempty[s]);
         mma_commit(&bars.pempty[pb]);
         if (t.last) mma_commit(&bars.ofull[t.ob]);
       };
@@ -349,7 +359,7 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
           for (int ks = 0; ks < D / 16; ++ks)
             mma_bf16(tmem + sb * HP, kd0 + uint64_t(((ks / 4) * TILE * 128 + (ks % 4) * 32) >> 4),
                      qd0 + uint64_t(((ks / 4) * HP * 128 + (ks % 4) * 32) >> 4), id_s, ks > 0 ? 1u : 0u);
-          mma_commit(&bars.kempty[s]);
+          if (C::NS != 2) mma_commit(&bars.kempty[s]);
           mma_commit(&bars.sfull[sb]);
           if (i == nt - 1) mma_commit(&bars.qempty[qb]);
           if (prev.valid) issue_pv(prev);

@@ -13,7 +13,6 @@ namespace hsa {
 namespace {
 
 constexpr int NT = 256;
-constexpr int NT_TOPK = 512;  // top-k rows hold up to m*B keys: 16 per thread at 8192
 
 // Kept-block list of one row: count of valid entries and candidate count
 // (tokens j <= t of the kept blocks). Returns false when the list does not
@@ -183,6 +182,153 @@ __global__ void __launch_bounds__(NT) topk_from_keys_kernel(RowMap rm, const int
   rs.compact(key, n, T, take_eq, [&](int rank, int c) { out[rank] = tok(c); });
 }
 
+// ---------------------------------------------------------------------------
+// Top-k with one warp per row (many rows): no CTA barriers. The warp streams
+// its row's keys (16-byte loads) once for min/max, once per 11-bit histogram
+// round into a warp-private 2048-bin shared histogram, and once to emit the
+// selected positions in ascending order.
+// ---------------------------------------------------------------------------
+constexpr int kWarpRowsPerCta = 8;
+constexpr int kWBins = 2048;
+
+// Calls f(key) for the keys [0, n) of `row`: 16-byte loads, lane-strided,
+// two 128-key steps in flight per iteration, scalar loads for the tail.
+template <class F>
+HSA_DEV void warp_stream_keys(const uint32_t* __restrict__ row, int n, F f) {
+  const int lane = threadIdx.x & 31;
+  const int n8 = n & ~255, n4 = n & ~127;
+  const uint4* r4 = reinterpret_cast<const uint4*>(row);
+  for (int c0 = 0; c0 < n8; c0 += 256) {
+    const uint4 a = __ldg(r4 + (c0 >> 2) + lane), b = __ldg(r4 + (c0 >> 2) + 32 + lane);
+    f(a.x); f(a.y); f(a.z); f(a.w); f(b.x); f(b.y); f(b.z); f(b.w);
+  }
+  if (n4 > n8) {
+    const uint4 a = __ldg(r4 + (n8 >> 2) + lane);
+    f(a.x); f(a.y); f(a.z); f(a.w);
+  }
+  for (int c = n4 + lane; c < n; c += 32) f(__ldg(row + c));
+}
+
+__global__ void __launch_bounds__(32 * kWarpRowsPerCta) topk_warp_rows_kernel(
+    RowMap rm, int64_t rows, const int32_t* __restrict__ blocks, const uint32_t* __restrict__ tkeys, int B,
+    int m, int k, int32_t* __restrict__ indices) {
+  extern __shared__ uint32_t wsm[];  // per warp: kWBins histogram bins, then 256 block ids
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t i = int64_t(blockIdx.x) * kWarpRowsPerCta + warp;
+  if (i >= rows) return;
+  uint32_t* hist = wsm + warp * (kWBins + 256);
+  int* blk = reinterpret_cast<int*>(hist + kWBins);
+  int32_t* out = indices + i * int64_t(k);
+  if (!rm.valid(i)) {
+    for (int s = lane; s < k; s += 32) out[s] = -1;
+    return;
+  }
+  const int64_t t = rm.pos(i);
+  for (int s = lane; s < m; s += 32) blk[s] = blocks[i * m + s];
+  __syncwarp();
+  int nblk = 0, n = 0;
+  const bool ok = row_candidates(blk, m, t, B, &nblk, &n);
+  if (!ok) {
+    for (int s = lane; s < k; s += 32) out[s] = -1;
+    return;
+  }
+  const bool pow2 = (B & (B - 1)) == 0;
+  const int lb = 31 - __clz(B);
+  auto tok = [&](int c) -> int32_t {
+    return pow2 ? (blk[c >> lb] << lb) + (c & (B - 1)) : int32_t(int64_t(blk[c / B]) * B + c % B);
+  };
+  if (n <= k) {
+    for (int s = lane; s < k; s += 32) out[s] = s < n ? tok(s) : -1;
+    return;
+  }
+  const uint32_t* row = tkeys + i * int64_t(m) * B;
+  // narrow to the k-th largest key, 11 bits per round from the top
+  // (rounds of 11, 11 and 10 bits; a bin taken whole ends the search early)
+  const uint32_t hi = 0xffffffffu;
+  uint32_t base = 0u, width = 0xffffffffu, T = 0;
+  int rem = k, take_eq = 0;
+  for (;;) {
+    const int bits = 32 - __clz(width);
+    const int shift = bits > 11 ? bits - 11 : 0;
+    for (int e = lane; e < kWBins; e += 32) hist[e] = 0;
+    __syncwarp();
+    warp_stream_keys(row, n, [&](uint32_t u) {
+      const uint32_t d = u - base;
+      if (d <= width) atomicAdd(&hist[d >> shift], 1u);
+    });
+    __syncwarp();
+    // lane l owns bins [64 l, 64 l + 64); counts above each lane's range
+    uint32_t tot = 0;
+    for (int e = 0; e < 64; ++e) tot += hist[lane * 64 + e];
+    uint32_t incl = tot;  // sum over lanes >= lane
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_down_sync(kFull, incl, o);
+      if (lane + o < 32) incl += y;
+    }
+    const uint32_t above = incl - tot;
+    int found_bin = -1;
+    uint32_t found_above = 0;
+    if (above < uint32_t(rem) && uint32_t(rem) <= incl) {
+      uint32_t a = above;
+      for (int e = 63; e >= 0; --e) {
+        const uint32_t c = hist[lane * 64 + e];
+        if (a + c >= uint32_t(rem)) { found_bin = lane * 64 + e; found_above = a; break; }
+        a += c;
+      }
+    }
+    const unsigned who = __ballot_sync(kFull, found_bin >= 0);
+    const int src = __ffs(who) - 1;
+    const uint32_t bin = uint32_t(__shfl_sync(kFull, found_bin, src));
+    rem -= int(__shfl_sync(kFull, found_above, src));
+    const bool whole = hist[bin] == uint32_t(rem);
+    base += bin << shift;
+    width = min(shift ? (1u << shift) - 1u : 0u, hi - base);
+    __syncwarp();
+    if (whole && base > 0u) { T = base - 1u; take_eq = 0; break; }
+    if (shift == 0) { T = base; take_eq = rem; break; }
+  }
+  // emit ascending: rank = (#keys > T before) + min(#keys == T before, take_eq)
+  int gt = 0, eq = 0;
+  const int n4 = n & ~127;
+  const unsigned below = (1u << lane) - 1u;
+  for (int c0 = 0; c0 < n4; c0 += 128) {
+    const int c = c0 + 4 * lane;
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(row + c));
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+    int g4 = 0, e4 = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) { g4 += u[e] > T; e4 += u[e] == T; }
+    // exclusive prefix of the lane counts
+    int gp = g4, ep = e4;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int yg = __shfl_up_sync(kFull, gp, o), ye = __shfl_up_sync(kFull, ep, o);
+      if (lane >= o) { gp += yg; ep += ye; }
+    }
+    int gb = gt + gp - g4, eb = eq + ep - e4;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (u[e] > T) { out[gb + min(eb, take_eq)] = tok(c + e); ++gb; }
+      else if (u[e] == T) { if (eb < take_eq) out[gb + eb] = tok(c + e); ++eb; }
+    }
+    gt += __shfl_sync(kFull, gp, 31);
+    eq += __shfl_sync(kFull, ep, 31);
+  }
+  for (int c0 = n4; c0 < n; c0 += 32) {
+    const int c = c0 + lane;
+    const uint32_t u = c < n ? __ldg(row + c) : 0u;
+    const unsigned bg = __ballot_sync(kFull, c < n && u > T);
+    const unsigned be = __ballot_sync(kFull, c < n && u == T);
+    const int gb = gt + __popc(bg & below), eb = eq + __popc(be & below);
+    if (c < n && u > T) out[gb + min(eb, take_eq)] = tok(c);
+    else if (c < n && u == T && eb < take_eq) out[gb + eb] = tok(c);
+    gt += __popc(bg);
+    eq += __popc(be);
+  }
+  (void)nblk;
+}
+
 }  // namespace
 
 // Keys per thread for up to n keys over NT threads: 1, 2, 4, ..., 64.
@@ -240,11 +386,11 @@ void launch_topk_from_keys(RowMap rm, int64_t rows, const int32_t* blocks, const
     HSA_KPT_DISPATCH(kpt, HSA_TOPK)
 #undef HSA_TOPK
   } else {
-#define HSA_TOPK(K) topk_from_keys_kernel<NT_TOPK, K><<<unsigned(rows), NT_TOPK, 0, s>>>(rm, blocks, tkeys, B, m, k, indices)
-    int kpt = 1;
-    while (int64_t(kpt) * NT_TOPK < int64_t(m) * B) kpt *= 2;
-    HSA_KPT_DISPATCH(kpt, HSA_TOPK)
-#undef HSA_TOPK
+    // many rows: one warp per row
+    const int smem = kWarpRowsPerCta * (kWBins + 256) * 4;
+    cudaFuncSetAttribute(topk_warp_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    topk_warp_rows_kernel<<<unsigned((rows + kWarpRowsPerCta - 1) / kWarpRowsPerCta), 32 * kWarpRowsPerCta, smem,
+                            s>>>(rm, rows, blocks, tkeys, B, m, k, indices);
   }
 }
 
