@@ -91,11 +91,7 @@ namespace {
 // failure, so one lost arrival cannot keep any warp spinning for long.
 HSA_DEV bool wait_bar(uint64_t* bar, uint32_t parity, bool& dead) {
   if (dead) return false;
-  for (uint32_t it = 0; it < (1u << 24); ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 4095u) == 4095u && *(volatile int*)&g_attn_err) { dead = true; return false; }
-  }
-  atomicExch(&g_attn_err, 1);
+  if (mbar_wait_bounded(bar, parity, &g_attn_err)) return true;
   dead = true;
   return false;
 }

@@ -36,15 +36,37 @@ HSA_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait: spins until the phase with `parity` completes or the
-// iteration limit is hit; on timeout sets *err (global) and returns false.
-// Callers then skip the dependent work and run to completion, so a lost
-// arrival can never hang the GPU.
-constexpr uint32_t kSpinLimit = 1u << 26;
-HSA_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, int* err, int code) {
-  for (uint32_t it = 0; it < kSpinLimit; ++it)
-    if (mbar_try_wait(bar, parity)) return true;
-  if (err) atomicExch(err, code);
+// try_wait with a suspend-time hint: while the phase is incomplete the
+// thread may sleep for up to `ns` nanoseconds, waking when the phase
+// completes, instead of coming straight back to probe again.
+HSA_DEV bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait on a phase. The first probe is a plain try_wait (a phase that
+// is already complete answers at once); later probes sleep, so waiting warps
+// do not take issue slots from the warps doing the work. Gives up after
+// kWaitCycles SM cycles (about two seconds), setting *err, or as soon as
+// another thread has set *err; returns whether the phase completed. Callers
+// then skip the dependent work and run to completion, so a lost arrival can
+// never hang the GPU.
+constexpr long long kWaitCycles = 1ll << 32;
+constexpr uint32_t kSuspendNs = 100000;
+HSA_DEV bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
+    if ((it & 15u) == 0 && *(volatile int*)err) return false;
+    if (clock64() - t0 > kWaitCycles) break;
+  }
+  atomicExch(err, 1);
   return false;
 }
 
