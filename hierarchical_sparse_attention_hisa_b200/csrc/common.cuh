@@ -37,6 +37,8 @@ HSA_DEV uint32_t score_key(float f) {
   if ((u << 1) == 0u) u = 0u;
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
+// The score a key stands for (inverse of score_key; -0 comes back as +0).
+HSA_DEV float key_score(uint32_t u) { return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u); }
 
 // Which absolute position a query row has, and where its sequence lives.
 // Prefill: one sequence, query row i is position Lk - Lq + i.
@@ -241,32 +243,25 @@ struct RegSelect {
     const int lane = threadIdx.x & 31;
     volatile int* s = scratch + NW + 2;  // [0] min, [1] max, [2] bin, [3] above
     const int p0 = threadIdx.x * KPT;
-    uint32_t lo = 0xffffffffu, hi = 0u;
+    // smallest and largest key for which in(key) holds, over the CTA
+    auto key_range = [&](auto in, uint32_t* lo_out, uint32_t* hi_out) {
+      uint32_t lo = 0xffffffffu, hi = 0u;
 #pragma unroll
-    for (int j = 0; j < KPT; ++j)
-      if (p0 + j < n) { lo = min(lo, key[j]); hi = max(hi, key[j]); }
-    lo = __reduce_min_sync(kFull, lo);
-    hi = __reduce_max_sync(kFull, hi);
-    if (threadIdx.x == 0) { s[0] = int(0xffffffffu); s[1] = 0; }
-    __syncthreads();
-    if (lane == 0) { atomicMin((unsigned*)&s[0], lo); atomicMax((unsigned*)&s[1], hi); }
-    __syncthreads();
-    const uint32_t kmax = uint32_t(s[1]);
-    uint32_t base = uint32_t(s[0]);
-    uint32_t width = kmax - base;
-    int rem = r;
-    for (;;) {
-      const int bits = 32 - __clz(width);
-      const int shift = bits > 11 ? bits - 11 : 0;
-#pragma unroll
-      for (int e = 0; e < BPT; ++e) hist[threadIdx.x * BPT + e] = 0;
+      for (int j = 0; j < KPT; ++j)
+        if (p0 + j < n && in(key[j])) { lo = min(lo, key[j]); hi = max(hi, key[j]); }
+      lo = __reduce_min_sync(kFull, lo);
+      hi = __reduce_max_sync(kFull, hi);
+      if (threadIdx.x == 0) { s[0] = int(0xffffffffu); s[1] = 0; }
       __syncthreads();
-#pragma unroll
-      for (int j = 0; j < KPT; ++j) {
-        const uint32_t d = key[j] - base;
-        if (p0 + j < n && d <= width) atomicAdd(&hist[d >> shift], 1u);
-      }
+      if (lane == 0) { atomicMin((unsigned*)&s[0], lo); atomicMax((unsigned*)&s[1], hi); }
       __syncthreads();
+      *lo_out = uint32_t(s[0]);
+      *hi_out = uint32_t(s[1]);
+      __syncthreads();
+    };
+    // the bin of `hist` that holds the rem-th largest counted key; rem
+    // becomes its rank inside that bin
+    auto pick = [&](int& rem) -> uint32_t {
       uint32_t cnt[BPT], tot = 0;
 #pragma unroll
       for (int e = 0; e < BPT; ++e) { cnt[e] = hist[threadIdx.x * BPT + e]; tot += cnt[e]; }
@@ -281,8 +276,53 @@ struct RegSelect {
         }
       }
       __syncthreads();
-      const uint32_t bin = uint32_t(s[2]);
       rem -= s[3];
+      return uint32_t(s[2]);
+    };
+    uint32_t base, kmax;
+    key_range([](uint32_t) { return true; }, &base, &kmax);
+    int rem = r;
+    // First round over bins linear in the score value. Keys are the
+    // order-preserving images of fp32 scores; bins on their top bits would
+    // crowd a row into the few bins that span its exponents, while linear
+    // bins spread it over all of them. The bin floor((x - lo) * c), in
+    // round-to-nearest fp32, never decreases as x grows, so every bin is a
+    // contiguous key range and the rounds below can continue inside it.
+    // Rows whose range is not finite skip this round.
+    const float flo = key_score(base), fhi = key_score(kmax);
+    const float c = float(kBins) / (fhi - flo);
+    if (flo < fhi && c > 0.f && c < INFINITY) {
+      auto vbin = [&](uint32_t u) { return min(uint32_t(kBins - 1), __float2uint_rz((key_score(u) - flo) * c)); };
+#pragma unroll
+      for (int e = 0; e < BPT; ++e) hist[threadIdx.x * BPT + e] = 0;
+      __syncthreads();
+#pragma unroll
+      for (int j = 0; j < KPT; ++j)
+        if (p0 + j < n) atomicAdd(&hist[vbin(key[j])], 1u);
+      __syncthreads();
+      const uint32_t bin = pick(rem);
+      const bool whole = hist[bin] == uint32_t(rem);
+      key_range([&](uint32_t u) { return vbin(u) == bin; }, &base, &kmax);
+      if (whole && base > 0u) {
+        *T_out = base - 1u;
+        *take_eq = 0;
+        return;
+      }
+    }
+    uint32_t width = kmax - base;
+    for (;;) {
+      const int bits = 32 - __clz(width);
+      const int shift = bits > 11 ? bits - 11 : 0;
+#pragma unroll
+      for (int e = 0; e < BPT; ++e) hist[threadIdx.x * BPT + e] = 0;
+      __syncthreads();
+#pragma unroll
+      for (int j = 0; j < KPT; ++j) {
+        const uint32_t d = key[j] - base;
+        if (p0 + j < n && d <= width) atomicAdd(&hist[d >> shift], 1u);
+      }
+      __syncthreads();
+      const uint32_t bin = pick(rem);
       const bool whole = hist[bin] == uint32_t(rem);  // every key of the bin is taken
       base += bin << shift;
       width = min(shift ? (1u << shift) - 1u : 0u, kmax - base);

@@ -8,6 +8,7 @@
 //   top-k tokens   (section 第二步): from the token-score keys of one row,
 //                  candidates enumerated in ascending token order.
 #include "kernels.cuh"
+#include "tc.cuh"
 
 namespace hsa {
 namespace {
@@ -329,6 +330,236 @@ __global__ void __launch_bounds__(32 * kWarpRowsPerCta) topk_warp_rows_kernel(
   (void)nblk;
 }
 
+// One row per 256-thread CTA (m*B <= 8192, a multiple of 4): the row's keys
+// are staged once in shared memory and every pass reads them from there.
+// Thread t owns positions [32 t, 32 t + 32) as eight 16-byte chunks whose
+// slots are XOR-swizzled, so that the coalesced fill and a warp reading one
+// chunk of each of its threads are both free of bank conflicts.
+// The threshold is located first in 2048 bins linear in the score value
+// (bins on key bits would crowd a row into the few bins of its exponent
+// range). A value bin is a contiguous key range, found exactly by bisection
+// of the bin function, and usually holds a handful of keys, which are
+// gathered and ranked directly. A crowded bin, or a row whose score range is
+// not finite, continues with 11-bit rounds on the key bits.
+constexpr int kRowNT = 256, kRowCap = 8192, kRowKPT = kRowCap / kRowNT, kRowChunks = kRowKPT / 4;
+constexpr int kRowBins = 2048, kRowBPT = kRowBins / kRowNT;
+constexpr int kRowRank = 64;  // largest threshold bin ranked pairwise
+static_assert(kRowChunks == 8, "chunk swizzle assumes eight chunks per thread");
+
+struct RowSmem {
+  uint4 keys[kRowCap / 4];
+  uint32_t hist[kRowBins];
+  uint32_t list[kRowRank];
+  int blk[256];
+  int sc[16];
+  uint32_t red[32];  // [0..7] minima, [8..15] maxima, [16] list count, [17] T, [18] take_eq, [19..20] bin range
+  int pk[2];
+};
+
+HSA_DEV int row_slot(int g) { return (g & ~7) | ((g & 7) ^ ((g >> 3) & 7)); }
+
+__global__ void __launch_bounds__(kRowNT) topk_rows_kernel(RowMap rm, const int32_t* __restrict__ blocks,
+                                                           const uint32_t* __restrict__ tkeys, int B, int m,
+                                                           int k, int32_t* __restrict__ indices) {
+  extern __shared__ __align__(16) uint8_t row_smem_raw[];
+  RowSmem& S = *reinterpret_cast<RowSmem*>(row_smem_raw);
+  const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
+  const int64_t i = blockIdx.x;
+  int32_t* out = indices + i * int64_t(k);
+  if (!rm.valid(i)) {
+    for (int s = tid; s < k; s += kRowNT) out[s] = -1;
+    return;
+  }
+  const int64_t t = rm.pos(i);
+  for (int s = tid; s < m; s += kRowNT) S.blk[s] = blocks[i * m + s];
+  for (int e = 0; e < kRowBPT; ++e) S.hist[tid * kRowBPT + e] = 0;
+  if (tid == 0) {
+    int nblk = 0, ncand = 0;
+    const bool ok = row_candidates(S.blk, m, t, B, &nblk, &ncand);
+    S.pk[0] = ok ? ncand : -1;
+    S.red[16] = 0;
+  }
+  __syncthreads();
+  const int n = S.pk[0];
+  if (n < 0) {
+    for (int s = tid; s < k; s += kRowNT) out[s] = -1;
+    return;
+  }
+  const bool pow2 = (B & (B - 1)) == 0;
+  const int lb = 31 - __clz(B);
+  auto tok = [&](int c) -> int32_t {
+    return pow2 ? (S.blk[c >> lb] << lb) + (c & (B - 1)) : int32_t(int64_t(S.blk[c / B]) * B + c % B);
+  };
+  if (n <= k) {
+    for (int s = tid; s < k; s += kRowNT) out[s] = s < n ? tok(s) : -1;
+    return;
+  }
+  {
+    const int nslot4 = (m * B) >> 2;
+    const uint4* src = reinterpret_cast<const uint4*>(tkeys + i * int64_t(m) * B);
+    for (int g = tid; g < nslot4; g += kRowNT) tc::cp_async16(tc::smem_u32(&S.keys[row_slot(g)]), src + g);
+    tc::cp_async_wait_all();
+    __syncthreads();
+  }
+  const int p0 = tid * kRowKPT;
+  const int lim = n - p0;  // key j of this thread is a candidate iff j < lim
+  auto chunk = [&](int c) { return S.keys[(tid << 3) | (c ^ (tid & 7))]; };
+  // runs f(j, key) over this thread's candidates, in position order
+  auto each = [&](auto f) {
+#pragma unroll 2
+    for (int c = 0; c < kRowChunks; ++c) {
+      if (4 * c >= lim) break;
+      const uint4 v = chunk(c);
+      f(4 * c, v.x);
+      if (4 * c + 1 < lim) f(4 * c + 1, v.y);
+      if (4 * c + 2 < lim) f(4 * c + 2, v.z);
+      if (4 * c + 3 < lim) f(4 * c + 3, v.w);
+    }
+  };
+  auto block_min_max = [&](uint32_t lo, uint32_t hi, uint32_t* lo_out, uint32_t* hi_out) {
+    lo = __reduce_min_sync(kFull, lo);
+    hi = __reduce_max_sync(kFull, hi);
+    if (l == 0) { S.red[w] = lo; S.red[8 + w] = hi; }
+    __syncthreads();
+    lo = S.red[0]; hi = S.red[8];
+#pragma unroll
+    for (int u = 1; u < kRowNT / 32; ++u) { lo = min(lo, S.red[u]); hi = max(hi, S.red[8 + u]); }
+    *lo_out = lo; *hi_out = hi;
+  };
+  // the bin of `hist` holding the rem-th largest counted key; rem becomes the
+  // rank inside that bin
+  auto pick = [&](int& rem) -> uint32_t {
+    uint32_t cnt[kRowBPT], tot = 0;
+#pragma unroll
+    for (int e = 0; e < kRowBPT; e += 4) {
+      const uint4 h4 = *reinterpret_cast<const uint4*>(&S.hist[tid * kRowBPT + e]);
+      cnt[e] = h4.x; cnt[e + 1] = h4.y; cnt[e + 2] = h4.z; cnt[e + 3] = h4.w;
+      tot += h4.x + h4.y + h4.z + h4.w;
+    }
+    int total;
+    const int above = block_exclusive_scan_rev<kRowNT>(int(tot), S.sc, &total);
+    if (uint32_t(above) < uint32_t(rem) && uint32_t(rem) <= uint32_t(above) + tot) {
+      uint32_t a = uint32_t(above);
+#pragma unroll
+      for (int e = kRowBPT - 1; e >= 0; --e) {
+        if (a + cnt[e] >= uint32_t(rem)) { S.pk[0] = tid * kRowBPT + e; S.pk[1] = int(a); break; }
+        a += cnt[e];
+      }
+    }
+    __syncthreads();
+    rem -= S.pk[1];
+    return uint32_t(S.pk[0]);
+  };
+
+  uint32_t ulo, uhi;
+  {
+    uint32_t lo = 0xffffffffu, hi = 0u;
+    each([&](int, uint32_t u) { lo = min(lo, u); hi = max(hi, u); });
+    block_min_max(lo, hi, &ulo, &uhi);
+  }
+  int rem = k;
+  uint32_t T = 0;
+  int take_eq = 0;
+  int ngt = 0, neq = 0;  // this thread's keys above T and equal to T
+  bool counted = false;
+  const float flo = key_score(ulo), fhi = key_score(uhi);
+  const float c = float(kRowBins) / (fhi - flo);
+  if (flo < fhi && c > 0.f && c < INFINITY) {
+    // floor((x - lo) * c) in round-to-nearest fp32 never decreases as x grows
+    auto vbin = [&](uint32_t u) { return min(uint32_t(kRowBins - 1), __float2uint_rz((key_score(u) - flo) * c)); };
+    each([&](int, uint32_t u) { atomicAdd(&S.hist[vbin(u)], 1u); });
+    __syncthreads();
+    const uint32_t bin = pick(rem);
+    const uint32_t cstar = S.hist[bin];
+    if (tid < 2) {
+      // smallest key of bin (tid 0) or of the next bin (tid 1), by bisection
+      const uint32_t target = bin + uint32_t(tid);
+      uint32_t a = ulo, z = uhi;  // answer in (a, z] unless vbin(a) >= target
+      if (vbin(a) >= target) {
+        z = a;
+      } else {
+        while (z - a > 1u) {
+          const uint32_t mid = a + (z - a) / 2u;
+          if (vbin(mid) >= target) z = mid; else a = mid;
+        }
+      }
+      S.red[19 + tid] = (tid == 1 && vbin(uhi) < target) ? uhi + 1u : z;  // bin + 1 past the top: end
+    }
+    __syncthreads();
+    const uint32_t blo = S.red[19], bhi = S.red[20] - 1u;  // the bin's keys: [blo, bhi]
+    if (cstar <= uint32_t(kRowRank)) {
+      uint32_t mine = 0;  // this thread's keys inside the bin
+      each([&](int j, uint32_t u) {
+        if (u > bhi) ++ngt;
+        else if (u >= blo) { S.list[atomicAdd(&S.red[16], 1u)] = u; mine |= 1u << j; }
+      });
+      __syncthreads();
+      if (tid < int(cstar)) {
+        const uint32_t x = S.list[tid];
+        int gt = 0, ge = 0;
+        for (int b = 0; b < int(cstar); ++b) {
+          const uint32_t y = S.list[b];
+          gt += y > x;
+          ge += y >= x;
+        }
+        if (gt < rem && rem <= ge) { S.red[17] = x; S.red[18] = uint32_t(rem - gt); }  // writers agree
+      }
+      __syncthreads();
+      T = S.red[17];
+      take_eq = int(S.red[18]);
+      while (mine) {
+        const int j = __ffs(mine) - 1;
+        mine &= mine - 1u;
+        const uint4 v = chunk(j >> 2);
+        const uint32_t u = (j & 3) == 0 ? v.x : (j & 3) == 1 ? v.y : (j & 3) == 2 ? v.z : v.w;
+        ngt += u > T;
+        neq += u == T;
+      }
+      counted = true;
+    } else {
+      ulo = blo;
+      uhi = bhi;
+    }
+  }
+  if (!counted) {
+    // 11-bit rounds over the key range [ulo, uhi] that holds the threshold
+    uint32_t base = ulo, width = uhi - ulo;
+    for (;;) {
+      const int bits = 32 - __clz(width);
+      const int shift = bits > 11 ? bits - 11 : 0;
+      for (int e = 0; e < kRowBPT; ++e) S.hist[tid * kRowBPT + e] = 0;
+      __syncthreads();
+      each([&](int, uint32_t u) {
+        const uint32_t d = u - base;
+        if (d <= width) atomicAdd(&S.hist[d >> shift], 1u);
+      });
+      __syncthreads();
+      const uint32_t bin = pick(rem);
+      const bool whole = S.hist[bin] == uint32_t(rem);
+      base += bin << shift;
+      width = min(shift ? (1u << shift) - 1u : 0u, uhi - base);
+      __syncthreads();
+      if (whole && base > 0u) { T = base - 1u; take_eq = 0; break; }
+      if (shift == 0) { T = base; take_eq = rem; break; }
+    }
+    each([&](int, uint32_t u) { ngt += u > T; neq += u == T; });
+  }
+  // emit in position order: slot = (#keys > T before) + min(#keys == T before, take_eq)
+  int total;
+  const int before = block_exclusive_scan<kRowNT>((ngt << 16) | neq, S.sc, &total);  // both < 2^15
+  int G = before >> 16, Q = before & 0xffff;
+  each([&](int j, uint32_t u) {
+    if (u < T) return;
+    if (u > T) {
+      out[G + min(Q, take_eq)] = tok(p0 + j);
+      ++G;
+    } else {
+      if (Q < take_eq) out[G + Q] = tok(p0 + j);
+      ++Q;
+    }
+  });
+}
+
 }  // namespace
 
 // Keys per thread for up to n keys over NT threads: 1, 2, 4, ..., 64.
@@ -385,8 +616,13 @@ void launch_topk_from_keys(RowMap rm, int64_t rows, const int32_t* blocks, const
     while (int64_t(kpt) * 1024 < int64_t(m) * B) kpt *= 2;
     HSA_KPT_DISPATCH(kpt, HSA_TOPK)
 #undef HSA_TOPK
+  } else if (int64_t(m) * B <= kRowCap && (int64_t(m) * B) % 4 == 0 && m <= 256 &&
+             (reinterpret_cast<uintptr_t>(tkeys) & 15u) == 0) {
+    // many rows of up to 8192 candidates: a 128-thread CTA per row, keys in registers
+    cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sizeof(RowSmem)));
+    topk_rows_kernel<<<unsigned(rows), kRowNT, sizeof(RowSmem), s>>>(rm, blocks, tkeys, B, m, k, indices);
   } else {
-    // many rows: one warp per row
+    // many longer rows: one warp per row
     const int smem = kWarpRowsPerCta * (kWBins + 256) * 4;
     cudaFuncSetAttribute(topk_warp_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     topk_warp_rows_kernel<<<unsigned((rows + kWarpRowsPerCta - 1) / kWarpRowsPerCta), 32 * kWarpRowsPerCta, smem,

@@ -120,6 +120,27 @@ def test_index_all_ties_goes_to_lowest_indices(hsa):
     assert np.array_equal(got, oracle.index(q, kk, 32, 6, 50))
 
 
+@pytest.mark.parametrize("probs,k", [
+    ({1.0: 0.5}, 512),            # two score values: the threshold bin holds ~1000 tied keys
+    ({3.0: 0.2, 2.0: 0.02}, 430),  # the threshold usually falls among ~40 tied keys of value 2
+])
+def test_index_few_score_values_ties_exact(hsa, probs, k):
+    # every score is k[:, 0] (q is all ones, the other key dims are 0), so most
+    # candidates tie and selection inside the tied group goes by lowest index
+    rng = np.random.default_rng(16)
+    Lq = Lk = 4096
+    q = synth.f32_to_bf16_bits(np.ones((Lq, 64), np.float32))
+    vals = np.zeros((Lk, 64), np.float32)
+    u = rng.random(Lk)
+    lo = 0.0
+    for v, pr in probs.items():
+        vals[(u >= lo) & (u < lo + pr), 0] = v
+        lo += pr
+    kk = synth.f32_to_bf16_bits(vals)
+    got = run_index(hsa, q, kk, 128, 16, k)
+    assert np.array_equal(got, oracle.index(q, kk, 128, 16, k))
+
+
 def test_index_extreme_magnitudes_exact(hsa):
     # all entries +-8: token scores reach +-8192 and block scores +-2^20
     rng = np.random.default_rng(15)
