@@ -371,16 +371,20 @@ __global__ void __launch_bounds__(kRowNT) topk_rows_kernel(RowMap rm, const int3
     return;
   }
   const int64_t t = rm.pos(i);
-  for (int s = tid; s < m; s += kRowNT) S.blk[s] = blocks[i * m + s];
+  // the kept-block list (m <= kRowNT entries): leading entries >= 0,
+  // ascending, the query's own block last
+  const int bk = tid < m ? blocks[i * m + tid] : -1;
+  if (tid < m) S.blk[tid] = bk;
   for (int e = 0; e < kRowBPT; ++e) S.hist[tid * kRowBPT + e] = 0;
-  if (tid == 0) {
-    int nblk = 0, ncand = 0;
-    const bool ok = row_candidates(S.blk, m, t, B, &nblk, &ncand);
-    S.pk[0] = ok ? ncand : -1;
-    S.red[16] = 0;
-  }
+  if (tid == 0) { S.pk[0] = m; S.red[16] = 0; }
   __syncthreads();
-  const int n = S.pk[0];
+  if (tid < m && bk < 0) atomicMin(&S.pk[0], tid);
+  __syncthreads();
+  const int nblk = S.pk[0];
+  const bool unordered = tid + 1 < nblk && bk >= S.blk[tid + 1];
+  int n = -1;
+  if (!__syncthreads_or(unordered) && nblk > 0 && S.blk[nblk - 1] == int(t / B))
+    n = int((nblk - 1) * int64_t(B) + (t - int64_t(S.blk[nblk - 1]) * B + 1));
   if (n < 0) {
     for (int s = tid; s < k; s += kRowNT) out[s] = -1;
     return;
@@ -465,33 +469,21 @@ __global__ void __launch_bounds__(kRowNT) topk_rows_kernel(RowMap rm, const int3
   const float flo = key_score(ulo), fhi = key_score(uhi);
   const float c = float(kRowBins) / (fhi - flo);
   if (flo < fhi && c > 0.f && c < INFINITY) {
-    // floor((x - lo) * c) in round-to-nearest fp32 never decreases as x grows
-    auto vbin = [&](uint32_t u) { return min(uint32_t(kRowBins - 1), __float2uint_rz((key_score(u) - flo) * c)); };
+    // the bin fma(x, c, -lo * c), rounded to nearest and truncated, never
+    // decreases as x grows
+    const float nb = -flo * c;
+    auto vbin = [&](uint32_t u) { return min(uint32_t(kRowBins - 1), __float2uint_rz(fmaf(key_score(u), c, nb))); };
     each([&](int, uint32_t u) { atomicAdd(&S.hist[vbin(u)], 1u); });
     __syncthreads();
     const uint32_t bin = pick(rem);
     const uint32_t cstar = S.hist[bin];
-    if (tid < 2) {
-      // smallest key of bin (tid 0) or of the next bin (tid 1), by bisection
-      const uint32_t target = bin + uint32_t(tid);
-      uint32_t a = ulo, z = uhi;  // answer in (a, z] unless vbin(a) >= target
-      if (vbin(a) >= target) {
-        z = a;
-      } else {
-        while (z - a > 1u) {
-          const uint32_t mid = a + (z - a) / 2u;
-          if (vbin(mid) >= target) z = mid; else a = mid;
-        }
-      }
-      S.red[19 + tid] = (tid == 1 && vbin(uhi) < target) ? uhi + 1u : z;  // bin + 1 past the top: end
-    }
-    __syncthreads();
-    const uint32_t blo = S.red[19], bhi = S.red[20] - 1u;  // the bin's keys: [blo, bhi]
     if (cstar <= uint32_t(kRowRank)) {
+      // gather the bin and rank it pairwise: T is its rem-th largest key
       uint32_t mine = 0;  // this thread's keys inside the bin
       each([&](int j, uint32_t u) {
-        if (u > bhi) ++ngt;
-        else if (u >= blo) { S.list[atomicAdd(&S.red[16], 1u)] = u; mine |= 1u << j; }
+        const uint32_t b = vbin(u);
+        ngt += b > bin;
+        if (b == bin) { S.list[atomicAdd(&S.red[16], 1u)] = u; mine |= 1u << j; }
       });
       __syncthreads();
       if (tid < int(cstar)) {
@@ -517,8 +509,13 @@ __global__ void __launch_bounds__(kRowNT) topk_rows_kernel(RowMap rm, const int3
       }
       counted = true;
     } else {
-      ulo = blo;
-      uhi = bhi;
+      // a crowded bin: its key range, then rounds on the key bits inside it
+      uint32_t lo = 0xffffffffu, hi = 0u;
+      each([&](int, uint32_t u) {
+        if (vbin(u) == bin) { lo = min(lo, u); hi = max(hi, u); }
+      });
+      __syncthreads();  // every thread has read hist[bin] and red[] before they are reused
+      block_min_max(lo, hi, &ulo, &uhi);
     }
   }
   if (!counted) {
@@ -544,20 +541,33 @@ __global__ void __launch_bounds__(kRowNT) topk_rows_kernel(RowMap rm, const int3
     }
     each([&](int, uint32_t u) { ngt += u > T; neq += u == T; });
   }
-  // emit in position order: slot = (#keys > T before) + min(#keys == T before, take_eq)
-  int total;
-  const int before = block_exclusive_scan<kRowNT>((ngt << 16) | neq, S.sc, &total);  // both < 2^15
-  int G = before >> 16, Q = before & 0xffff;
-  each([&](int j, uint32_t u) {
-    if (u < T) return;
-    if (u > T) {
-      out[G + min(Q, take_eq)] = tok(p0 + j);
-      ++G;
-    } else {
-      if (Q < take_eq) out[G + Q] = tok(p0 + j);
-      ++Q;
+  // emit in position order: slot = (#keys > T before) + min(#keys == T before, take_eq).
+  // Warp w emits positions [1024 w, 1024 w + 1024) (its threads' keys), 32 at
+  // a time, one per lane, with ballot prefix counts.
+  {
+    const int wsum = __reduce_add_sync(kFull, (ngt << 16) | neq);  // per warp < 2^11 of each
+    if (l == 0) S.red[w] = uint32_t(wsum);
+    __syncthreads();
+    int G = 0, Q = 0;
+    for (int u = 0; u < w; ++u) { G += int(S.red[u] >> 16); Q += int(S.red[u] & 0xffffu); }
+    const unsigned below = (1u << l) - 1u;
+    const int lane_word = l & 3, lane_chunk = l >> 2;
+    const int wend = min(1024, n - 1024 * w);  // candidates of this warp
+    const uint32_t* kw = reinterpret_cast<const uint32_t*>(S.keys);
+    for (int s0 = 0; s0 < wend; s0 += 32) {
+      const int tt = 32 * w + (s0 >> 5);  // owner thread of these 32 positions
+      const int p = 1024 * w + s0 + l;
+      const uint32_t u = kw[4 * ((tt << 3) | (lane_chunk ^ (tt & 7))) + lane_word];
+      const bool in = s0 + l < wend;
+      const bool gt = in && u > T, eq = in && u == T;
+      const unsigned bg = __ballot_sync(kFull, gt), be = __ballot_sync(kFull, eq);
+      const int rg = G + __popc(bg & below), re = Q + __popc(be & below);
+      const int32_t tk = tok(p);
+      if (gt || (eq && re < take_eq)) out[rg + min(re, take_eq)] = tk;
+      G += __popc(bg);
+      Q += __popc(be);
     }
-  });
+  }
 }
 
 }  // namespace
