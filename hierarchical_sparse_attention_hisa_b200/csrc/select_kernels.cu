@@ -330,7 +330,7 @@ __global__ void __launch_bounds__(32 * kWarpRowsPerCta) topk_warp_rows_kernel(
   (void)nblk;
 }
 
-// One row per 256-thread CTA (m*B <= 8192, a multiple of 4): the row's keys
+// One row per 256-thread CTA (m*B <= 8192, B a power of two >= 4): the row's keys
 // are staged once in shared memory and every pass reads them from there.
 // Thread t owns positions [32 t, 32 t + 32) as eight 16-byte chunks whose
 // slots are XOR-swizzled, so that the coalesced fill and a warp reading one
@@ -358,7 +358,7 @@ struct RowSmem {
 
 HSA_DEV int row_slot(int g) { return (g & ~7) | ((g & 7) ^ ((g >> 3) & 7)); }
 
-__global__ void __launch_bounds__(kRowNT) topk_rows_kernel(RowMap rm, const int32_t* __restrict__ blocks,
+__global__ void __launch_bounds__(kRowNT, 4) topk_rows_kernel(RowMap rm, const int32_t* __restrict__ blocks,
                                                            const uint32_t* __restrict__ tkeys, int B, int m,
                                                            int k, int32_t* __restrict__ indices) {
   extern __shared__ __align__(16) uint8_t row_smem_raw[];
@@ -389,13 +389,9 @@ __global__ void __launch_bounds__(kRowNT) topk_rows_kernel(RowMap rm, const int3
     for (int s = tid; s < k; s += kRowNT) out[s] = -1;
     return;
   }
-  const bool pow2 = (B & (B - 1)) == 0;
-  const int lb = 31 - __clz(B);
-  auto tok = [&](int c) -> int32_t {
-    return pow2 ? (S.blk[c >> lb] << lb) + (c & (B - 1)) : int32_t(int64_t(S.blk[c / B]) * B + c % B);
-  };
+  const int lb = 31 - __clz(B);  // B is a power of two here
   if (n <= k) {
-    for (int s = tid; s < k; s += kRowNT) out[s] = s < n ? tok(s) : -1;
+    for (int s = tid; s < k; s += kRowNT) out[s] = s < n ? (S.blk[s >> lb] << lb) + (s & (B - 1)) : -1;
     return;
   }
   {
@@ -406,18 +402,22 @@ __global__ void __launch_bounds__(kRowNT) topk_rows_kernel(RowMap rm, const int3
     __syncthreads();
   }
   const int p0 = tid * kRowKPT;
-  const int lim = n - p0;  // key j of this thread is a candidate iff j < lim
+  const int nj = max(0, min(kRowKPT, n - p0));  // this thread's candidates: keys j < nj
   auto chunk = [&](int c) { return S.keys[(tid << 3) | (c ^ (tid & 7))]; };
-  // runs f(j, key) over this thread's candidates, in position order
+  auto key_at = [&](int j) {
+    const uint4 v = chunk(j >> 2);
+    return (j & 3) == 0 ? v.x : (j & 3) == 1 ? v.y : (j & 3) == 2 ? v.z : v.w;
+  };
+  // f(j, key) for all 32 keys of this thread (fully unrolled: j is a
+  // constant); f must ignore j >= nj
   auto each = [&](auto f) {
-#pragma unroll 2
+#pragma unroll
     for (int c = 0; c < kRowChunks; ++c) {
-      if (4 * c >= lim) break;
       const uint4 v = chunk(c);
       f(4 * c, v.x);
-      if (4 * c + 1 < lim) f(4 * c + 1, v.y);
-      if (4 * c + 2 < lim) f(4 * c + 2, v.z);
-      if (4 * c + 3 < lim) f(4 * c + 3, v.w);
+      f(4 * c + 1, v.y);
+      f(4 * c + 2, v.z);
+      f(4 * c + 3, v.w);
     }
   };
   auto block_min_max = [&](uint32_t lo, uint32_t hi, uint32_t* lo_out, uint32_t* hi_out) {
@@ -458,39 +458,51 @@ __global__ void __launch_bounds__(kRowNT) topk_rows_kernel(RowMap rm, const int3
   uint32_t ulo, uhi;
   {
     uint32_t lo = 0xffffffffu, hi = 0u;
-    each([&](int, uint32_t u) { lo = min(lo, u); hi = max(hi, u); });
+    each([&](int j, uint32_t u) {
+      if (j < nj) { lo = min(lo, u); hi = max(hi, u); }
+    });
     block_min_max(lo, hi, &ulo, &uhi);
   }
   int rem = k;
   uint32_t T = 0;
   int take_eq = 0;
-  int ngt = 0, neq = 0;  // this thread's keys above T and equal to T
-  bool counted = false;
+  uint32_t gtm = 0, eqm = 0;  // this thread's keys above T, and equal to T (bit j: key j)
+  bool done = false;
   const float flo = key_score(ulo), fhi = key_score(uhi);
   const float c = float(kRowBins) / (fhi - flo);
   if (flo < fhi && c > 0.f && c < INFINITY) {
     // the bin fma(x, c, -lo * c), rounded to nearest and truncated, never
     // decreases as x grows
     const float nb = -flo * c;
-    auto vbin = [&](uint32_t u) { return min(uint32_t(kRowBins - 1), __float2uint_rz(fmaf(key_score(u), c, nb))); };
-    each([&](int, uint32_t u) { atomicAdd(&S.hist[vbin(u)], 1u); });
+    uint32_t vbr[kRowKPT / 2];  // the bins of keys 2r and 2r + 1
+#pragma unroll
+    for (int r = 0; r < kRowKPT / 2; ++r) vbr[r] = 0;
+    each([&](int j, uint32_t u) {
+      const uint32_t b = min(uint32_t(kRowBins - 1), __float2uint_rz(fmaf(key_score(u), c, nb)));
+      if (j < nj) atomicAdd(&S.hist[b], 1u);
+      vbr[j >> 1] |= b << (16 * (j & 1));
+    });
     __syncthreads();
     const uint32_t bin = pick(rem);
     const uint32_t cstar = S.hist[bin];
+    uint32_t binm = 0;  // this thread's keys inside the bin
+#pragma unroll
+    for (int j = 0; j < kRowKPT; ++j) {
+      const uint32_t b = (vbr[j >> 1] >> (16 * (j & 1))) & 0xffffu;
+      if (j < nj) {
+        gtm |= uint32_t(b > bin) << j;
+        binm |= uint32_t(b == bin) << j;
+      }
+    }
     if (cstar <= uint32_t(kRowRank)) {
       // gather the bin and rank it pairwise: T is its rem-th largest key
-      uint32_t mine = 0;  // this thread's keys inside the bin
-      each([&](int j, uint32_t u) {
-        const uint32_t b = vbin(u);
-        ngt += b > bin;
-        if (b == bin) { S.list[atomicAdd(&S.red[16], 1u)] = u; mine |= 1u << j; }
-      });
+      for (uint32_t mm = binm; mm; mm &= mm - 1u) S.list[atomicAdd(&S.red[16], 1u)] = key_at(__ffs(mm) - 1);
       __syncthreads();
       if (tid < int(cstar)) {
         const uint32_t x = S.list[tid];
         int gt = 0, ge = 0;
-        for (int b = 0; b < int(cstar); ++b) {
-          const uint32_t y = S.list[b];
+        for (int q = 0; q < int(cstar); ++q) {
+          const uint32_t y = S.list[q];
           gt += y > x;
           ge += y >= x;
         }
@@ -499,26 +511,26 @@ __global__ void __launch_bounds__(kRowNT) topk_rows_kernel(RowMap rm, const int3
       __syncthreads();
       T = S.red[17];
       take_eq = int(S.red[18]);
-      while (mine) {
-        const int j = __ffs(mine) - 1;
-        mine &= mine - 1u;
-        const uint4 v = chunk(j >> 2);
-        const uint32_t u = (j & 3) == 0 ? v.x : (j & 3) == 1 ? v.y : (j & 3) == 2 ? v.z : v.w;
-        ngt += u > T;
-        neq += u == T;
+      for (uint32_t mm = binm; mm; mm &= mm - 1u) {
+        const int j = __ffs(mm) - 1;
+        const uint32_t u = key_at(j);
+        gtm |= uint32_t(u > T) << j;
+        eqm |= uint32_t(u == T) << j;
       }
-      counted = true;
+      done = true;
     } else {
       // a crowded bin: its key range, then rounds on the key bits inside it
       uint32_t lo = 0xffffffffu, hi = 0u;
-      each([&](int, uint32_t u) {
-        if (vbin(u) == bin) { lo = min(lo, u); hi = max(hi, u); }
-      });
-      __syncthreads();  // every thread has read hist[bin] and red[] before they are reused
+      for (uint32_t mm = binm; mm; mm &= mm - 1u) {
+        const uint32_t u = key_at(__ffs(mm) - 1);
+        lo = min(lo, u);
+        hi = max(hi, u);
+      }
+      __syncthreads();  // every thread has read hist[bin] before red[] and hist are reused
       block_min_max(lo, hi, &ulo, &uhi);
     }
   }
-  if (!counted) {
+  if (!done) {
     // 11-bit rounds over the key range [ulo, uhi] that holds the threshold
     uint32_t base = ulo, width = uhi - ulo;
     for (;;) {
@@ -526,9 +538,9 @@ __global__ void __launch_bounds__(kRowNT) topk_rows_kernel(RowMap rm, const int3
       const int shift = bits > 11 ? bits - 11 : 0;
       for (int e = 0; e < kRowBPT; ++e) S.hist[tid * kRowBPT + e] = 0;
       __syncthreads();
-      each([&](int, uint32_t u) {
+      each([&](int j, uint32_t u) {
         const uint32_t d = u - base;
-        if (d <= width) atomicAdd(&S.hist[d >> shift], 1u);
+        if (j < nj && d <= width) atomicAdd(&S.hist[d >> shift], 1u);
       });
       __syncthreads();
       const uint32_t bin = pick(rem);
@@ -539,33 +551,27 @@ __global__ void __launch_bounds__(kRowNT) topk_rows_kernel(RowMap rm, const int3
       if (whole && base > 0u) { T = base - 1u; take_eq = 0; break; }
       if (shift == 0) { T = base; take_eq = rem; break; }
     }
-    each([&](int, uint32_t u) { ngt += u > T; neq += u == T; });
+    gtm = eqm = 0;
+    each([&](int j, uint32_t u) {
+      if (j < nj) {
+        gtm |= uint32_t(u > T) << j;
+        eqm |= uint32_t(u == T) << j;
+      }
+    });
   }
-  // emit in position order: slot = (#keys > T before) + min(#keys == T before, take_eq).
-  // Warp w emits positions [1024 w, 1024 w + 1024) (its threads' keys), 32 at
-  // a time, one per lane, with ballot prefix counts.
-  {
-    const int wsum = __reduce_add_sync(kFull, (ngt << 16) | neq);  // per warp < 2^11 of each
-    if (l == 0) S.red[w] = uint32_t(wsum);
-    __syncthreads();
-    int G = 0, Q = 0;
-    for (int u = 0; u < w; ++u) { G += int(S.red[u] >> 16); Q += int(S.red[u] & 0xffffu); }
-    const unsigned below = (1u << l) - 1u;
-    const int lane_word = l & 3, lane_chunk = l >> 2;
-    const int wend = min(1024, n - 1024 * w);  // candidates of this warp
-    const uint32_t* kw = reinterpret_cast<const uint32_t*>(S.keys);
-    for (int s0 = 0; s0 < wend; s0 += 32) {
-      const int tt = 32 * w + (s0 >> 5);  // owner thread of these 32 positions
-      const int p = 1024 * w + s0 + l;
-      const uint32_t u = kw[4 * ((tt << 3) | (lane_chunk ^ (tt & 7))) + lane_word];
-      const bool in = s0 + l < wend;
-      const bool gt = in && u > T, eq = in && u == T;
-      const unsigned bg = __ballot_sync(kFull, gt), be = __ballot_sync(kFull, eq);
-      const int rg = G + __popc(bg & below), re = Q + __popc(be & below);
-      const int32_t tk = tok(p);
-      if (gt || (eq && re < take_eq)) out[rg + min(re, take_eq)] = tk;
-      G += __popc(bg);
-      Q += __popc(be);
+  // emit in position order: slot = (#keys > T before) + min(#keys == T before, take_eq)
+  int total;
+  const int before = block_exclusive_scan<kRowNT>((__popc(gtm) << 16) | __popc(eqm), S.sc, &total);  // < 2^14 each
+  int G = before >> 16, Q = before & 0xffff;
+  for (uint32_t mm = gtm | eqm; mm; mm &= mm - 1u) {
+    const int j = __ffs(mm) - 1;
+    const int32_t tk = (S.blk[(p0 + j) >> lb] << lb) + ((p0 + j) & (B - 1));
+    if ((gtm >> j) & 1u) {
+      out[G + min(Q, take_eq)] = tk;
+      ++G;
+    } else {
+      if (Q < take_eq) out[G + Q] = tk;
+      ++Q;
     }
   }
 }
@@ -626,7 +632,7 @@ void launch_topk_from_keys(RowMap rm, int64_t rows, const int32_t* blocks, const
     while (int64_t(kpt) * 1024 < int64_t(m) * B) kpt *= 2;
     HSA_KPT_DISPATCH(kpt, HSA_TOPK)
 #undef HSA_TOPK
-  } else if (int64_t(m) * B <= kRowCap && (int64_t(m) * B) % 4 == 0 && m <= 256 &&
+  } else if (int64_t(m) * B <= kRowCap && (B & (B - 1)) == 0 && B >= 4 && m <= 256 &&
              (reinterpret_cast<uintptr_t>(tkeys) & 15u) == 0) {
     // many rows of up to 8192 candidates: a 128-thread CTA per row, keys in registers
     cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sizeof(RowSmem)));
