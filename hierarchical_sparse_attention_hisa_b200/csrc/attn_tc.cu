@@ -330,10 +330,11 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
         const uint64_t a0 = smem_desc(smem_u32(sm + C::OFF_V + s * C::KV_BYTES), TILE * 128, 1024, kSw128);
         const uint64_t b0 = smem_desc(smem_u32(sm + C::OFF_P + pb * C::P_BYTES), 16384, 8 * C::P_ROW, C::P_SWZ);
         const uint32_t d = tmem + 2 * HP + t.ob * HP;
+        const uint32_t alo = uint32_t(a0), ahi = uint32_t(a0 >> 32), blo = uint32_t(b0), bhi = uint32_t(b0 >> 32);
 #pragma unroll
         for (int ks = 0; ks < TILE / 16; ++ks)
-          mma_bf16(d, a0 + uint64_t((ks * 2048) >> 4), b0 + uint64_t((ks * 16 * C::P_ROW) >> 4), id_o,
-                   (t.first && ks == 0) ? 0u : 1u);
+          mma_bf16_split(d, alo + ((ks * 2048) >> 4), ahi, blo + ((ks * 16 * C::P_ROW) >> 4), bhi, id_o,
+                         (t.first && ks == 0) ? 0u : 1u);
         if (C::NS != 2) mma_commit(&bars.vempty[s]);
         mma_commit(&bars.pempty[pb]);
         if (t.last) mma_commit(&bars.ofull[t.ob]);
@@ -345,16 +346,18 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
         if (nt == 0) { mbar_arrive(&bars.qempty[qb]); continue; }
         const uint32_t ob = oq & 1;
         const uint64_t qd0 = smem_desc(smem_u32(sm + C::OFF_Q + qb * C::Q_BYTES), 16, 1024, kSw128);
+        const uint32_t qlo = uint32_t(qd0), qhi = uint32_t(qd0 >> 32);
         for (int i = 0; i < nt && !dead; ++i, ++g) {
           const int s = g % C::NS, sb = g & 1;
           if (!wait_bar(&bars.kfull[s], (g / C::NS) & 1, dead)) break;
           if (!wait_bar(&bars.sempty[sb], ((g >> 1) & 1) ^ 1, dead)) break;
           tc_fence_after();
           const uint64_t kd0 = smem_desc(smem_u32(sm + C::OFF_K + s * C::KV_BYTES), 16, 1024, kSw128);
+          const uint32_t klo = uint32_t(kd0), khi = uint32_t(kd0 >> 32);
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks)
-            mma_bf16(tmem + sb * HP, kd0 + uint64_t(((ks / 4) * TILE * 128 + (ks % 4) * 32) >> 4),
-                     qd0 + uint64_t(((ks / 4) * HP * 128 + (ks % 4) * 32) >> 4), id_s, ks > 0 ? 1u : 0u);
+            mma_bf16_split(tmem + sb * HP, klo + (((ks / 4) * TILE * 128 + (ks % 4) * 32) >> 4), khi,
+                           qlo + (((ks / 4) * HP * 128 + (ks % 4) * 32) >> 4), qhi, id_s, ks > 0 ? 1u : 0u);
           if (C::NS != 2) mma_commit(&bars.kempty[s]);
           mma_commit(&bars.sfull[sb]);
           if (i == nt - 1) mma_commit(&bars.qempty[qb]);
