@@ -121,6 +121,31 @@ def pinned_bf16(u16):
     return t.pin_memory()
 
 
+# DRAM traffic of the sparse-attention kernel from one ncu capture (the
+# 8192-query case of `bench.py --profile-case attn_last8k`, summarised in
+# profiles/sparse_attn_tc_prefill64k_last8k.md): dram__bytes_read.sum +
+# dram__bytes_write.sum of one launch. Q, O and the index rows scale with the
+# queries; the K/V cache (read once) does not. The figure belongs to the
+# kernel sources it was captured from and is reported only while they are
+# unchanged.
+ATTN_CAPTURE = {"queries": 8192, "read": 235.910656e6, "write": 121.618688e6, "sources": "93a2fab279aebe56"}
+ATTN_SOURCES = ("csrc/attn_tc.cu", "csrc/tc.cuh", "csrc/common.cuh")
+
+
+def attn_traffic(Lq, L, d):
+    import hashlib
+    h = hashlib.sha256()
+    pkg = os.path.join(ROOT, "hierarchical_sparse_attention_hisa_b200")
+    for f in ATTN_SOURCES:
+        with open(os.path.join(pkg, f), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest()[:16] != ATTN_CAPTURE["sources"]:
+        return None
+    kv = 2.0 * L * d * 2
+    per_q = (ATTN_CAPTURE["read"] + ATTN_CAPTURE["write"] - kv) / ATTN_CAPTURE["queries"]
+    return per_q * Lq + kv
+
+
 def attn_flops(idx_counts, H, d):
     # QK^T and PV: 2 * 2 * H * d multiply-adds per kept (query, key) pair
     return 4.0 * H * d * float(idx_counts)
@@ -236,7 +261,8 @@ def bench_hsa(args, rank, world, device):
                    "l2": "flushed (512 MiB write) between timed steps"},
         "breakdown_ms": {"hsa_index": sum(t_index) / args.steps, "hsa_sparse_attn": attn_ms},
         "roofline": {"kernel": "sparse attention", "bound": "tensor", "achieved": achieved,
-                     "peak": tf, "unit": "TFLOP/s", "frac": achieved / tf, "traffic": None,
+                     "peak": tf, "unit": "TFLOP/s", "frac": achieved / tf,
+                     "traffic": attn_traffic(w.Lq, w.L, w.d),
                      "peak_source": f"{src} bf16 burst",
                      "flops_per_launch": flops},
         "gpu_launches": int(launches),
