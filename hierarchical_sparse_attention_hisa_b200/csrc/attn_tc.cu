@@ -426,21 +426,31 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.sempty[sb]);
-        bool mine = false;
+        // x becomes the exponent scale * s - m; a row without a valid key and
+        // padded heads get -inf (no weight)
         const bool live = oks && valid;
+        float tmax = -INFINITY;
 #pragma unroll
         for (int h = 0; h < HH; ++h) {
-          x[h] = (live && h0 + h < H) ? x[h] * scale_log2 : -INFINITY;
-          mine |= x[h] - m[h] > kRescaleThreshold;
+          x[h] = fmaf(x[h], scale_log2, -m[h]);
+          tmax = fmaxf(tmax, x[h]);
         }
-        mine |= !complete;
+        if (!live || h0 + HH > H) {
+          tmax = -INFINITY;
+#pragma unroll
+          for (int h = 0; h < HH; ++h) {
+            if (!live || h0 + h >= H) x[h] = -INFINITY;
+            tmax = fmaxf(tmax, x[h]);
+          }
+        }
+        const bool mine = tmax > kRescaleThreshold || !complete;
         dead = dead || !oks;
         if (wg_or(bar_id, i == 0 || mine || dead)) {
           if (wg_or(bar_id, dead)) { quit = true; break; }
           // raise the running maxima of this warpgroup's heads to cover the tile
 #pragma unroll
           for (int h = 0; h < HH; ++h) {
-            const float wm = redux_max(x[h]);
+            const float wm = redux_max(x[h] + m[h]);  // the tile's scaled scores
             if (lane == (h & 31)) red[wq][h0 + h] = wm;
           }
           wg_sync(bar_id);
@@ -456,7 +466,9 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
 #pragma unroll
           for (int h = 0; h < HH; ++h) {
             const float n = mh[h0 + h];
-            m[h] = n == -INFINITY ? 0.f : n;
+            const float mn = n == -INFINITY ? 0.f : n;
+            x[h] += m[h] - mn;  // re-centre the exponents on the new maximum
+            m[h] = mn;
             all = all && (n != -INFINITY || h0 + h >= H);
           }
           complete = all;
@@ -491,7 +503,7 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
         uint32_t w[(HH + 1) / 2];
 #pragma unroll
         for (int e = 0; e < HH / 2; ++e) {
-          const float p0 = ex2(x[2 * e] - m[2 * e]), p1 = ex2(x[2 * e + 1] - m[2 * e + 1]);
+          const float p0 = ex2(x[2 * e]), p1 = ex2(x[2 * e + 1]);
           lp[2 * e] += p0;
           lp[2 * e + 1] += p1;
           w[e] = cvt_bf16x2(p0, p1);
