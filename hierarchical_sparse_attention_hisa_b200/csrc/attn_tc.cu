@@ -64,6 +64,8 @@ struct Cfg {
 struct Bars {
   uint64_t kfull[3], kempty[3], vfull[3], vempty[3];
   uint64_t qfull[2], qempty[2], sfull[2], sempty[2], pfull[2], pempty[2], ofull[2], oempty[2];
+  // two stages: sgo = K tile landed + S buffer read, pgo = P tile written + V tile landed
+  uint64_t sgo[2], pgo[2];
   uint64_t done;
 };
 
@@ -214,6 +216,9 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
       mbar_init(&bars.qfull[b], 1); mbar_init(&bars.qempty[b], 1 + C::NSW);
       mbar_init(&bars.sfull[b], 1); mbar_init(&bars.sempty[b], C::NSW);
       mbar_init(&bars.pfull[b], C::NSW); mbar_init(&bars.pempty[b], 1);
+      mbar_init(&bars.sgo[b], NPW * 32 + C::NSW); mbar_init(&bars.pgo[b], NPW * 32 + C::NSW);
+      // each S buffer starts out read: credit the softmax arrivals of its first use
+      for (int u = 0; u < C::NSW; ++u) mbar_arrive(&bars.sgo[b]);
       mbar_init(&bars.ofull[b], 1); mbar_init(&bars.oempty[b], C::NSW);
     }
     mbar_init(&bars.done, 1);
@@ -300,13 +305,13 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
 #pragma unroll
         for (int u = 0; u < PER; ++u)
           if (p + u * PT < TILE * 16) cp_async16(kt + dst[u], Kq + jr[u]);
-        cp_async_arrive(&bars.kfull[s]);
+        cp_async_arrive(C::NS == 2 ? &bars.sgo[s] : &bars.kfull[s]);
         if (!wait_warp(C::NS == 2 ? &bars.pempty[s] : &bars.vempty[s], ph ^ 1, dead)) break;
         const uint32_t vt = smem_u32(sm + C::OFF_V + s * C::KV_BYTES);
 #pragma unroll
         for (int u = 0; u < PER; ++u)
           if (p + u * PT < TILE * 16) cp_async16(vt + dst[u], Vq + jr[u]);
-        cp_async_arrive(&bars.vfull[s]);
+        cp_async_arrive(C::NS == 2 ? &bars.pgo[s] : &bars.vfull[s]);
       }
     }
     cp_async_wait_all();  // every copy has landed before the CTA may exit
@@ -323,8 +328,13 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
       struct Pend { uint32_t g, ob, oq; bool first, last, valid; } prev{0, 0, 0, false, false, false};
       auto issue_pv = [&](const Pend& t) {
         const int pb = t.g & 1, s = t.g % C::NS;
-        if (!wait_bar(&bars.pfull[pb], (t.g >> 1) & 1, dead)) return;
-        if (!wait_bar(&bars.vfull[s], (t.g / C::NS) & 1, dead)) return;
+        if constexpr (C::NS == 2) {
+          // one wait per tile: P written and V landed
+          if (!wait_bar(&bars.pgo[pb], (t.g >> 1) & 1, dead)) return;
+        } else {
+          if (!wait_bar(&bars.pfull[pb], (t.g >> 1) & 1, dead)) return;
+          if (!wait_bar(&bars.vfull[s], (t.g / C::NS) & 1, dead)) return;
+        }
         if (t.first && !wait_bar(&bars.oempty[t.ob], ((t.oq >> 1) & 1) ^ 1, dead)) return;
         tc_fence_after();
         const uint64_t a0 = smem_desc(smem_u32(sm + C::OFF_V + s * C::KV_BYTES), TILE * 128, 1024, kSw128);
@@ -349,8 +359,13 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
         const uint32_t qlo = uint32_t(qd0), qhi = uint32_t(qd0 >> 32);
         for (int i = 0; i < nt && !dead; ++i, ++g) {
           const int s = g % C::NS, sb = g & 1;
-          if (!wait_bar(&bars.kfull[s], (g / C::NS) & 1, dead)) break;
-          if (!wait_bar(&bars.sempty[sb], ((g >> 1) & 1) ^ 1, dead)) break;
+          if constexpr (C::NS == 2) {
+            // one wait per tile: K landed and the S buffer read by the softmax
+            if (!wait_bar(&bars.sgo[sb], (g >> 1) & 1, dead)) break;
+          } else {
+            if (!wait_bar(&bars.kfull[s], (g / C::NS) & 1, dead)) break;
+            if (!wait_bar(&bars.sempty[sb], ((g >> 1) & 1) ^ 1, dead)) break;
+          }
           tc_fence_after();
           const uint64_t kd0 = smem_desc(smem_u32(sm + C::OFF_K + s * C::KV_BYTES), 16, 1024, kSw128);
           const uint32_t klo = uint32_t(kd0), khi = uint32_t(kd0 >> 32);
@@ -425,7 +440,8 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.sempty[sb]);
+        // (with two stages this arrival counts toward the buffer's next use)
+        if (lane == 0) mbar_arrive(C::NS == 2 ? &bars.sgo[sb] : &bars.sempty[sb]);
         // x becomes the exponent scale * s - m; a row without a valid key and
         // padded heads get -inf (no weight)
         const bool live = oks && valid;
@@ -522,7 +538,7 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.pfull[pb]);
+        if (lane == 0) mbar_arrive(C::NS == 2 ? &bars.pgo[pb] : &bars.pfull[pb]);
       }
       if (quit) break;
       // ---- epilogue: row sums, normalise O^T, write O[q][h][r] for this warpgroup's heads
