@@ -295,8 +295,9 @@ struct DecodeWs {
 DecodeWs decode_ws(const hsa_params* p, int32_t batch, int64_t capacity) {
   DecodeWs w{};
   const int tiles = (p->k + 127) / 128;
-  // enough parts per query to give every SM work at small batch
-  w.parts = batch > 0 ? std::max(1, std::min(tiles, 128 / std::max(1, int(batch)))) : 1;
+  // enough parts per query to give every SM work at small batch, at most 16
+  // (the combine kernel holds every part's values in registers)
+  w.parts = batch > 0 ? std::max(1, std::min(std::min(tiles, 16), 128 / std::max(1, int(batch)))) : 1;
   size_t o = 0;
   auto take = [&](size_t bytes) { const size_t at = o; o += align_up(bytes > 0 ? bytes : 1); return at; };
   w.blocks = take(size_t(batch) * p->m * 4);
@@ -350,29 +351,32 @@ int hsa_decode_step(const hsa_params* p, int32_t batch, int64_t capacity, int32_
   uint32_t* tkeys = reinterpret_cast<uint32_t*>(ws + w.tkeys);
   const int64_t nbc = capacity / p->B;
   hsa::RowMap rm{batch, capacity, ctx_len, capacity};
+  // The step's kernels are programmatic dependent launches: each may begin
+  // launching while its predecessor runs, and waits for it before touching
+  // memory (griddepcontrol), which hides the launch gaps of a short step.
   // 1. append the new token (and the block sum of a block it completes)
   hsa::launch_decode_append(batch, capacity, ctx_len, p->B, p->d_idx, p->d, k_idx_cache, K_cache,
                             V_cache, ksum_cache, k_idx_new, K_new, V_new, stream);
   // 2. block scores against the block-sum cache, top-m with the forced blocks
   hsa::launch_decode_block_scores(batch, capacity, ctx_len, p->B, p->m, p->d_idx, q_idx_new, ksum_cache,
                                   bkeys, nbc, stream);
-  hsa::launch_topm_from_keys(rm, batch, bkeys, nbc, p->B, p->m, nbc > 2 ? nbc - 2 : 1, blocks, stream);
+  hsa::launch_topm_from_keys(rm, batch, bkeys, nbc, p->B, p->m, nbc > 2 ? nbc - 2 : 1, blocks, stream, true);
   // 3. token scores inside the kept blocks, top-k
   hsa::launch_decode_token_scores(batch, capacity, ctx_len, p->B, p->m, p->d_idx, blocks, q_idx_new,
                                   k_idx_cache, tkeys, stream);
-  hsa::launch_topk_from_keys(rm, batch, blocks, tkeys, p->B, p->m, p->k, idx, stream);
+  hsa::launch_topk_from_keys(rm, batch, blocks, tkeys, p->B, p->m, p->k, idx, stream, true);
   // 4. attention over the kept tokens: parts of each query on the tensor cores, then combined
   if (hsa::tc_attn_supported(p->H, p->d, batch, capacity)) {
     float* opart = reinterpret_cast<float*>(ws + w.opart);
     float* mpart = reinterpret_cast<float*>(ws + w.mpart);
     float* lpart = reinterpret_cast<float*>(ws + w.lpart);
     if (!hsa::launch_sparse_attn_tc_split(batch, Q_new, K_cache, V_cache, idx, capacity, p->k, p->H,
-                                          softmax_scale(p), w.parts, opart, mpart, lpart, stream))
+                                          softmax_scale(p), w.parts, opart, mpart, lpart, stream, true))
       return HSA_ERR_CUDA;
     hsa::launch_decode_combine(batch, capacity, ctx_len, p->H, p->d, w.parts, opart, mpart, lpart, O, stream);
   } else {
     hsa::launch_sparse_attn_simple(rm, batch, Q_new, K_cache, V_cache, idx, p->k, p->H, p->d,
-                                   softmax_scale(p), O, stream);
+                                   softmax_scale(p), O, stream, true);
   }
   // 5. the sequences grow by one token
   hsa::launch_decode_advance(batch, capacity, ctx_len, stream);

@@ -14,6 +14,8 @@ __global__ void __launch_bounds__(128) sparse_attn_simple_kernel(
     RowMap rm, const uint16_t* __restrict__ Q, const uint16_t* __restrict__ K,
     const uint16_t* __restrict__ V, const int32_t* __restrict__ idx, int k, int H,
     float scale_log2, uint16_t* __restrict__ O) {
+  griddep_wait();
+  griddep_launch();
   constexpr int NT = 128, CH = 32, G = NT / D;
   extern __shared__ __align__(16) float sm[];
   float* Qs = sm;                       // [H][D]
@@ -119,29 +121,28 @@ __global__ void __launch_bounds__(128) sparse_attn_simple_kernel(
 template <int D, int HR>
 static void launch_simple(RowMap rm, int64_t rows, const void* Q, const void* K, const void* V,
                           const int32_t* idx, int k, int H, float scale_log2, void* O,
-                          cudaStream_t s) {
+                          cudaStream_t s, bool pdl) {
   const size_t smem = sizeof(float) * (size_t(H) * D + 32 * (D + 1) + 32 * D + size_t(H) * 32 + 3 * H);
   cudaFuncSetAttribute(sparse_attn_simple_kernel<D, HR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        int(smem));
-  sparse_attn_simple_kernel<D, HR><<<unsigned(rows), 128, smem, s>>>(
-      rm, (const uint16_t*)Q, (const uint16_t*)K, (const uint16_t*)V, idx, k, H, scale_log2,
-      (uint16_t*)O);
+  launch_kernel(pdl, sparse_attn_simple_kernel<D, HR>, unsigned(rows), 128, smem, s, rm, (const uint16_t*)Q,
+                (const uint16_t*)K, (const uint16_t*)V, idx, k, H, scale_log2, (uint16_t*)O);
 }
 
 void launch_sparse_attn_simple(RowMap rm, int64_t rows, const void* Q, const void* K, const void* V,
                                const int32_t* idx, int k, int H, int d, float scale, void* O,
-                               cudaStream_t s) {
+                               cudaStream_t s, bool pdl) {
   if (rows == 0) return;
   count_launches(1);
   const float sl2 = scale * 1.4426950408889634f;
   if (d == 128) {
-    if (H <= 16) launch_simple<128, 16>(rm, rows, Q, K, V, idx, k, H, sl2, O, s);
-    else if (H <= 64) launch_simple<128, 64>(rm, rows, Q, K, V, idx, k, H, sl2, O, s);
-    else launch_simple<128, 128>(rm, rows, Q, K, V, idx, k, H, sl2, O, s);
+    if (H <= 16) launch_simple<128, 16>(rm, rows, Q, K, V, idx, k, H, sl2, O, s, pdl);
+    else if (H <= 64) launch_simple<128, 64>(rm, rows, Q, K, V, idx, k, H, sl2, O, s, pdl);
+    else launch_simple<128, 128>(rm, rows, Q, K, V, idx, k, H, sl2, O, s, pdl);
   } else {
-    if (H <= 16) launch_simple<64, 8>(rm, rows, Q, K, V, idx, k, H, sl2, O, s);
-    else if (H <= 64) launch_simple<64, 32>(rm, rows, Q, K, V, idx, k, H, sl2, O, s);
-    else launch_simple<64, 64>(rm, rows, Q, K, V, idx, k, H, sl2, O, s);
+    if (H <= 16) launch_simple<64, 8>(rm, rows, Q, K, V, idx, k, H, sl2, O, s, pdl);
+    else if (H <= 64) launch_simple<64, 32>(rm, rows, Q, K, V, idx, k, H, sl2, O, s, pdl);
+    else launch_simple<64, 64>(rm, rows, Q, K, V, idx, k, H, sl2, O, s, pdl);
   }
 }
 

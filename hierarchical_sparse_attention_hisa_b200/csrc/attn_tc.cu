@@ -190,6 +190,8 @@ template <int HP, int NPW>
 __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_kernel(
     const __grid_constant__ CUtensorMap qmap, const uint16_t* __restrict__ K, const uint16_t* __restrict__ V,
     const AttnArgs a) {
+  griddep_wait();
+  griddep_launch();
   using C = Cfg<HP, NPW>;
   const int32_t* __restrict__ idx = a.idx;
   const int Lk = a.Lk, k = a.k, H = a.H;
@@ -597,7 +599,7 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
 constexpr int kProducerWarps = 7;
 
 template <int HP>
-bool launch_hp(const void* Q, const void* K, const void* V, const AttnArgs& a, cudaStream_t s) {
+bool launch_hp(const void* Q, const void* K, const void* V, const AttnArgs& a, cudaStream_t s, bool pdl) {
   CUtensorMap qm;
   if (!make_tmap_2d(&qm, Q, uint64_t(a.Lq) * a.H, D, HP)) return false;
   using C = Cfg<HP, kProducerWarps>;
@@ -606,15 +608,16 @@ bool launch_hp(const void* Q, const void* K, const void* V, const AttnArgs& a, c
     return false;
   const int64_t items = int64_t(a.Lq) * a.items_per_query;
   const int grid = int(items < num_sms() ? items : num_sms());
-  kern<<<grid, 32 * C::NWARPS, C::SMEM, s>>>(qm, static_cast<const uint16_t*>(K), static_cast<const uint16_t*>(V), a);
+  launch_kernel(pdl, kern, grid, 32 * C::NWARPS, C::SMEM, s, qm, static_cast<const uint16_t*>(K),
+                static_cast<const uint16_t*>(V), a);
   return true;
 }
 
-bool launch_args(const void* Q, const void* K, const void* V, const AttnArgs& a, cudaStream_t s) {
+bool launch_args(const void* Q, const void* K, const void* V, const AttnArgs& a, cudaStream_t s, bool pdl) {
   count_launches(1);
-  if (a.H <= 16) return launch_hp<16>(Q, K, V, a, s);
-  if (a.H <= 32) return launch_hp<32>(Q, K, V, a, s);
-  return launch_hp<64>(Q, K, V, a, s);
+  if (a.H <= 16) return launch_hp<16>(Q, K, V, a, s, pdl);
+  if (a.H <= 32) return launch_hp<32>(Q, K, V, a, s, pdl);
+  return launch_hp<64>(Q, K, V, a, s, pdl);
 }
 
 }  // namespace
@@ -636,12 +639,12 @@ bool launch_sparse_attn_tc(int64_t Lq, const void* Q, const void* K, const void*
   a.items_per_query = 1;
   a.tiles_per_item = (k + TILE - 1) / TILE;
   a.O = static_cast<uint16_t*>(O);
-  return launch_args(Q, K, V, a, s);
+  return launch_args(Q, K, V, a, s, false);
 }
 
 bool launch_sparse_attn_tc_split(int batch, const void* Q, const void* Kc, const void* Vc, const int32_t* idx,
                                  int64_t capacity, int k, int H, float scale, int parts, float* Opart,
-                                 float* mpart, float* lpart, cudaStream_t s) {
+                                 float* mpart, float* lpart, cudaStream_t s, bool pdl) {
   if (batch == 0) return true;
   AttnArgs a{};
   a.idx = idx; a.Lq = batch; a.Lk = int(capacity); a.k = k; a.H = H;
@@ -651,7 +654,7 @@ bool launch_sparse_attn_tc_split(int batch, const void* Q, const void* Kc, const
   a.tiles_per_item = ((k + TILE - 1) / TILE + parts - 1) / parts;
   a.O = nullptr;
   a.Opart = Opart; a.mpart = mpart; a.lpart = lpart;
-  return launch_args(Q, Kc, Vc, a, s);
+  return launch_args(Q, Kc, Vc, a, s, pdl);
 }
 
 }  // namespace hsa

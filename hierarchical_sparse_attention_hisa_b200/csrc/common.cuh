@@ -38,6 +38,15 @@ HSA_DEV uint32_t score_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 // The score a key stands for (inverse of score_key; -0 comes back as +0).
+// Programmatic dependent launch. A kernel launched with the attribute may
+// start while the previous kernel of its stream is still running; it calls
+// griddep_wait() before touching any memory that kernel reads or writes (the
+// wait returns once that kernel has completed and its writes are visible; it
+// is a no-op for a normal launch), then griddep_launch() to let the next
+// kernel of the stream start its own launch.
+HSA_DEV void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+HSA_DEV void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 HSA_DEV float key_score(uint32_t u) { return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u); }
 
 // Which absolute position a query row has, and where its sequence lives.

@@ -11,6 +11,8 @@ __global__ void __launch_bounds__(128) decode_append_kernel(
     uint16_t* __restrict__ K_cache, uint16_t* __restrict__ V_cache, float* __restrict__ ksum_cache,
     const uint16_t* __restrict__ k_idx_new, const uint16_t* __restrict__ K_new,
     const uint16_t* __restrict__ V_new) {
+  griddep_wait();
+  griddep_launch();
   const int64_t b = blockIdx.x;
   const int64_t t = ctx[b];
   if (t < 0 || t >= capacity) return;
@@ -45,6 +47,8 @@ __global__ void __launch_bounds__(256) decode_block_scores_kernel(const int32_t*
                                                                   const uint16_t* __restrict__ q_new,
                                                                   const float* __restrict__ ksum_cache,
                                                                   uint32_t* __restrict__ bkeys, int64_t ld) {
+  griddep_wait();
+  griddep_launch();
   constexpr int VPL = DI / 32;  // fp32 values per lane
   const int64_t b = blockIdx.x;
   const int64_t t = ctx[b];
@@ -87,6 +91,8 @@ __global__ void __launch_bounds__(128) decode_token_scores_kernel(const int32_t*
                                                                   const uint16_t* __restrict__ q_new,
                                                                   const uint16_t* __restrict__ k_idx_cache,
                                                                   uint32_t* __restrict__ tkeys) {
+  griddep_wait();
+  griddep_launch();
   constexpr int LPR = DI / 8;          // lanes per row (8 bf16 each)
   constexpr int RPW = 32 / LPR;        // rows per warp instruction
   const int64_t b = blockIdx.x;
@@ -101,21 +107,29 @@ __global__ void __launch_bounds__(128) decode_token_scores_kernel(const int32_t*
   const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
   const uint16_t* kb = k_idx_cache + (b * capacity + int64_t(blk) * B) * DI;
   uint32_t* out = tkeys + (b * m + s) * int64_t(B);
-  for (int r0 = warp * RPW; r0 < B; r0 += 4 * RPW) {
-    const int r = r0 + rsub;
-    float acc = 0.f;
-    if (r < B) {
-      const uint4 kv = __ldg(reinterpret_cast<const uint4*>(kb + int64_t(r) * DI) + sub);
-      const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+  // eight rows per lane group in flight before any of them is reduced
+  constexpr int U = 8;
+  for (int r0 = warp * RPW; r0 < B; r0 += 4 * RPW * U) {
+    uint4 kv[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int r = r0 + u * 4 * RPW + rsub;
+      kv[u] = r < B ? __ldg(reinterpret_cast<const uint4*>(kb + int64_t(r) * DI) + sub) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int r = r0 + u * 4 * RPW + rsub;
+      const uint32_t kw[4] = {kv[u].x, kv[u].y, kv[u].z, kv[u].w};
+      float acc = 0.f;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         acc = __fmaf_rn(bf16_lo(qw[e]), bf16_lo(kw[e]), acc);
         acc = __fmaf_rn(bf16_hi(qw[e]), bf16_hi(kw[e]), acc);
       }
-    }
 #pragma unroll
-    for (int o = LPR / 2; o >= 1; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
-    if (sub == 0 && r < B) out[r] = score_key(acc);
+      for (int o = LPR / 2; o >= 1; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
+      if (sub == 0 && r < B) out[r] = score_key(acc);
+    }
   }
 }
 
@@ -125,24 +139,37 @@ __global__ void __launch_bounds__(128) decode_token_scores_kernel(const int32_t*
 __global__ void decode_combine_kernel(const int32_t* __restrict__ ctx, int64_t capacity, int H, int D, int parts,
                                       const float* __restrict__ Opart, const float* __restrict__ mpart,
                                       const float* __restrict__ lpart, uint16_t* __restrict__ O) {
+  griddep_wait();
+  griddep_launch();
   const int64_t b = blockIdx.x / H;
   const int h = blockIdx.x % H;
+  // every load issued before any is used: the sequence length, each part's
+  // maximum, row sum and output element
+  constexpr int PMAX = 16;
   const int64_t t = ctx[b];
+  float lv[PMAX], mv[PMAX], ov[PMAX];
+#pragma unroll
+  for (int p = 0; p < PMAX; ++p) {
+    if (p < parts) {
+      const int64_t w = b * parts + p;
+      lv[p] = lpart[w * H + h];
+      mv[p] = mpart[w * H + h];
+      ov[p] = Opart[(w * H + h) * D + threadIdx.x];
+    }
+  }
   float out = 0.f;
   if (t >= 0 && t < capacity) {
     float M = -INFINITY;
-    for (int p = 0; p < parts; ++p) {
-      const int64_t w = b * parts + p;
-      if (lpart[w * H + h] > 0.f) M = fmaxf(M, mpart[w * H + h]);
-    }
+#pragma unroll
+    for (int p = 0; p < PMAX; ++p)
+      if (p < parts && lv[p] > 0.f) M = fmaxf(M, mv[p]);
     float num = 0.f, den = 0.f;
-    for (int p = 0; p < parts; ++p) {
-      const int64_t w = b * parts + p;
-      const float l = lpart[w * H + h];
-      if (l > 0.f) {
-        const float f = exp2f(mpart[w * H + h] - M);
-        num = __fmaf_rn(f, Opart[(w * H + h) * D + threadIdx.x], num);
-        den = __fmaf_rn(f, l, den);
+#pragma unroll
+    for (int p = 0; p < PMAX; ++p) {
+      if (p < parts && lv[p] > 0.f) {
+        const float f = exp2f(mv[p] - M);
+        num = __fmaf_rn(f, ov[p], num);
+        den = __fmaf_rn(f, lv[p], den);
       }
     }
     out = den > 0.f ? num / den : 0.f;
@@ -159,11 +186,11 @@ void launch_decode_block_scores(int batch, int64_t capacity, const int32_t* ctx,
   const dim3 grid((unsigned)batch, (unsigned)((nbmax + per_cta - 1) / per_cta));
   count_launches(1);
   if (d_idx == 128)
-    decode_block_scores_kernel<128><<<grid, 256, 0, s>>>(ctx, capacity, B, m, per_cta, (const uint16_t*)q_new,
-                                                         ksum_cache, bkeys, ld);
+    launch_kernel(true, decode_block_scores_kernel<128>, grid, 256, 0, s, ctx, capacity, B, m, per_cta,
+                  (const uint16_t*)q_new, ksum_cache, bkeys, ld);
   else
-    decode_block_scores_kernel<64><<<grid, 256, 0, s>>>(ctx, capacity, B, m, per_cta, (const uint16_t*)q_new,
-                                                        ksum_cache, bkeys, ld);
+    launch_kernel(true, decode_block_scores_kernel<64>, grid, 256, 0, s, ctx, capacity, B, m, per_cta,
+                  (const uint16_t*)q_new, ksum_cache, bkeys, ld);
 }
 
 void launch_decode_token_scores(int batch, int64_t capacity, const int32_t* ctx, int B, int m, int d_idx,
@@ -173,22 +200,24 @@ void launch_decode_token_scores(int batch, int64_t capacity, const int32_t* ctx,
   const dim3 grid((unsigned)batch, (unsigned)m);
   count_launches(1);
   if (d_idx == 128)
-    decode_token_scores_kernel<128><<<grid, 128, 0, s>>>(ctx, capacity, B, m, blocks, (const uint16_t*)q_new,
-                                                         (const uint16_t*)k_idx_cache, tkeys);
+    launch_kernel(true, decode_token_scores_kernel<128>, grid, 128, 0, s, ctx, capacity, B, m, blocks,
+                  (const uint16_t*)q_new, (const uint16_t*)k_idx_cache, tkeys);
   else
-    decode_token_scores_kernel<64><<<grid, 128, 0, s>>>(ctx, capacity, B, m, blocks, (const uint16_t*)q_new,
-                                                        (const uint16_t*)k_idx_cache, tkeys);
+    launch_kernel(true, decode_token_scores_kernel<64>, grid, 128, 0, s, ctx, capacity, B, m, blocks,
+                  (const uint16_t*)q_new, (const uint16_t*)k_idx_cache, tkeys);
 }
 
 void launch_decode_combine(int batch, int64_t capacity, const int32_t* ctx, int H, int d, int parts,
                            const float* Opart, const float* mpart, const float* lpart, void* O, cudaStream_t s) {
   if (batch == 0) return;
   count_launches(1);
-  decode_combine_kernel<<<unsigned(batch * H), d, 0, s>>>(ctx, capacity, H, d, parts, Opart, mpart, lpart,
-                                                         (uint16_t*)O);
+  launch_kernel(true, decode_combine_kernel, unsigned(batch * H), d, 0, s, ctx, capacity, H, d, parts, Opart, mpart,
+                lpart, (uint16_t*)O);
 }
 
 __global__ void decode_advance_kernel(int batch, int64_t capacity, int32_t* ctx) {
+  griddep_wait();
+  griddep_launch();
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b < batch && ctx[b] >= 0 && ctx[b] < capacity) ctx[b] += 1;
 }
@@ -200,9 +229,9 @@ void launch_decode_append(int batch, int64_t capacity, const int32_t* ctx, int B
   if (batch == 0) return;
   count_launches(1);
 #define HSA_APPEND(DI, DA)                                                                      \
-  decode_append_kernel<DI, DA><<<batch, 128, 0, s>>>(                                           \
-      capacity, ctx, B, (uint16_t*)k_idx_cache, (uint16_t*)K_cache, (uint16_t*)V_cache,          \
-      ksum_cache, (const uint16_t*)k_idx_new, (const uint16_t*)K_new, (const uint16_t*)V_new)
+  launch_kernel(true, decode_append_kernel<DI, DA>, batch, 128, 0, s, capacity, ctx, B,           \
+                (uint16_t*)k_idx_cache, (uint16_t*)K_cache, (uint16_t*)V_cache, ksum_cache,       \
+                (const uint16_t*)k_idx_new, (const uint16_t*)K_new, (const uint16_t*)V_new)
   if (d_idx == 128 && d == 128) HSA_APPEND(128, 128);
   else if (d_idx == 128) HSA_APPEND(128, 64);
   else if (d == 128) HSA_APPEND(64, 128);
@@ -213,7 +242,7 @@ void launch_decode_append(int batch, int64_t capacity, const int32_t* ctx, int B
 void launch_decode_advance(int batch, int64_t capacity, int32_t* ctx, cudaStream_t s) {
   if (batch == 0) return;
   count_launches(1);
-  decode_advance_kernel<<<(batch + 127) / 128, 128, 0, s>>>(batch, capacity, ctx);
+  launch_kernel(true, decode_advance_kernel, (batch + 127) / 128, 128, 0, s, batch, capacity, ctx);
 }
 
 }  // namespace hsa

@@ -12,6 +12,24 @@ namespace hsa {
 // Counts kernel launches made by this library (see hsa_kernel_launches).
 void count_launches(int n);
 
+// Launches kern<<<grid, block, smem, s>>>(args...); with pdl set, as a
+// programmatic dependent launch (the kernel must begin with griddep_wait()).
+template <typename... KArgs, typename... Args>
+inline void launch_kernel(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                          Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  (void)cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // 2-D row-major bf16 [rows][cols] TMA map, box {64 columns, box_rows rows},
 // 128-byte swizzle. False if the driver entry point or the encoding fails.
 bool make_tmap_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
@@ -27,7 +45,7 @@ void launch_select_tokens(RowMap rm, int64_t rows, const void* q_idx, const void
                           cudaStream_t s);
 void launch_sparse_attn_simple(RowMap rm, int64_t rows, const void* Q, const void* K, const void* V,
                                const int32_t* idx, int k, int H, int d, float scale, void* O,
-                               cudaStream_t s);
+                               cudaStream_t s, bool pdl = false);
 // Tensor-core sparse attention (d = 128, 1 <= H <= 64); returns false if a
 // tensor map or launch attribute could not be set up.
 bool tc_attn_supported(int H, int d, int64_t Lq, int64_t Lk);
@@ -40,12 +58,12 @@ bool launch_token_score_gemm(const void* q_idx, const void* k_idx, int64_t Lq, i
                              int d_idx, const int4* tiles, const int* ntiles, const uint32_t* pairs,
                              int64_t max_tiles, uint32_t* out, cudaStream_t s);
 void launch_topm_from_keys(RowMap rm, int64_t rows, const uint32_t* bkeys, int64_t ld, int B, int m,
-                           int64_t max_cand, int32_t* blocks, cudaStream_t s);
+                           int64_t max_cand, int32_t* blocks, cudaStream_t s, bool pdl = false);
 void launch_pair_lists(RowMap rm, int64_t rows, const int32_t* blocks, int B, int m, int k, int nbins,
                        int* cnt, int* off, int* cursor, int4* tiles, int* ntiles, uint32_t* pairs,
                        cudaStream_t s);
 void launch_topk_from_keys(RowMap rm, int64_t rows, const int32_t* blocks, const uint32_t* tkeys, int B,
-                           int m, int k, int32_t* indices, cudaStream_t s);
+                           int m, int k, int32_t* indices, cudaStream_t s, bool pdl = false);
 void launch_decode_append(int batch, int64_t capacity, const int32_t* ctx, int B, int d_idx, int d,
                           void* k_idx_cache, void* K_cache, void* V_cache, float* ksum_cache,
                           const void* k_idx_new, const void* K_new, const void* V_new,
@@ -60,7 +78,7 @@ void launch_decode_combine(int batch, int64_t capacity, const int32_t* ctx, int 
                            const float* Opart, const float* mpart, const float* lpart, void* O, cudaStream_t s);
 bool launch_sparse_attn_tc_split(int batch, const void* Q, const void* Kc, const void* Vc, const int32_t* idx,
                                  int64_t capacity, int k, int H, float scale, int parts, float* Opart,
-                                 float* mpart, float* lpart, cudaStream_t s);
+                                 float* mpart, float* lpart, cudaStream_t s, bool pdl = false);
 void launch_decode_advance(int batch, int64_t capacity, int32_t* ctx, cudaStream_t s);
 
 }  // namespace hsa

@@ -32,6 +32,8 @@ HSA_DEV bool row_candidates(const int32_t* blk, int m, int64_t t, int B, int* nb
 template <int KPT>
 __global__ void __launch_bounds__(NT) topm_from_keys_kernel(RowMap rm, const uint32_t* __restrict__ bkeys,
                                                            int64_t ld, int B, int m, int32_t* __restrict__ blocks) {
+  griddep_wait();
+  griddep_launch();
   __shared__ uint32_t hist[RegSelect<NT, KPT>::kBins];
   __shared__ int scratch[NT / 32 + 8];
   const int64_t i = blockIdx.x;
@@ -140,6 +142,8 @@ template <int NT, int KPT>
 __global__ void __launch_bounds__(NT) topk_from_keys_kernel(RowMap rm, const int32_t* __restrict__ blocks,
                                                            const uint32_t* __restrict__ tkeys, int B, int m,
                                                            int k, int32_t* __restrict__ indices) {
+  griddep_wait();
+  griddep_launch();
   __shared__ uint32_t hist[RegSelect<NT, KPT>::kBins];
   __shared__ int scratch[NT / 32 + 8];
   __shared__ int blk[256];
@@ -361,6 +365,8 @@ HSA_DEV int row_slot(int g) { return (g & ~7) | ((g & 7) ^ ((g >> 3) & 7)); }
 __global__ void __launch_bounds__(kRowNT, 4) topk_rows_kernel(RowMap rm, const int32_t* __restrict__ blocks,
                                                            const uint32_t* __restrict__ tkeys, int B, int m,
                                                            int k, int32_t* __restrict__ indices) {
+  griddep_wait();
+  griddep_launch();
   extern __shared__ __align__(16) uint8_t row_smem_raw[];
   RowSmem& S = *reinterpret_cast<RowSmem*>(row_smem_raw);
   const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
@@ -597,10 +603,10 @@ static int keys_per_thread(int64_t n) {
   }
 
 void launch_topm_from_keys(RowMap rm, int64_t rows, const uint32_t* bkeys, int64_t ld, int B, int m,
-                           int64_t max_cand, int32_t* blocks, cudaStream_t s) {
+                           int64_t max_cand, int32_t* blocks, cudaStream_t s, bool pdl) {
   if (rows == 0) return;
   count_launches(1);
-#define HSA_TOPM(K) topm_from_keys_kernel<K><<<unsigned(rows), NT, 0, s>>>(rm, bkeys, ld, B, m, blocks)
+#define HSA_TOPM(K) launch_kernel(pdl, topm_from_keys_kernel<K>, unsigned(rows), NT, 0, s, rm, bkeys, ld, B, m, blocks)
   HSA_KPT_DISPATCH(keys_per_thread(max_cand), HSA_TOPM)
 #undef HSA_TOPM
 }
@@ -621,22 +627,23 @@ void launch_pair_lists(RowMap rm, int64_t rows, const int32_t* blocks, int B, in
 }
 
 void launch_topk_from_keys(RowMap rm, int64_t rows, const int32_t* blocks, const uint32_t* tkeys, int B,
-                           int m, int k, int32_t* indices, cudaStream_t s) {
+                           int m, int k, int32_t* indices, cudaStream_t s, bool pdl) {
   if (rows == 0) return;
   count_launches(1);
-  // few rows (a decode batch): wide CTAs cut each row's latency; many rows:
-  // 512 threads keep several CTAs per SM
-  if (rows < 2 * num_sms()) {
-#define HSA_TOPK(K) topk_from_keys_kernel<1024, K><<<unsigned(rows), 1024, 0, s>>>(rm, blocks, tkeys, B, m, k, indices)
+  if (int64_t(m) * B <= kRowCap && (B & (B - 1)) == 0 && B >= 4 && m <= 256 &&
+      (reinterpret_cast<uintptr_t>(tkeys) & 15u) == 0) {
+    // rows of up to 8192 candidates: a 256-thread CTA per row, the row staged in shared memory
+    cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sizeof(RowSmem)));
+    launch_kernel(pdl, topk_rows_kernel, unsigned(rows), kRowNT, sizeof(RowSmem), s, rm, blocks, tkeys, B, m, k,
+                  indices);
+  } else if (rows < 2 * num_sms()) {
+    // few longer rows (a decode batch): wide CTAs cut each row's latency
+#define HSA_TOPK(K) \
+  launch_kernel(pdl, topk_from_keys_kernel<1024, K>, unsigned(rows), 1024, 0, s, rm, blocks, tkeys, B, m, k, indices)
     int kpt = 1;
     while (int64_t(kpt) * 1024 < int64_t(m) * B) kpt *= 2;
     HSA_KPT_DISPATCH(kpt, HSA_TOPK)
 #undef HSA_TOPK
-  } else if (int64_t(m) * B <= kRowCap && (B & (B - 1)) == 0 && B >= 4 && m <= 256 &&
-             (reinterpret_cast<uintptr_t>(tkeys) & 15u) == 0) {
-    // many rows of up to 8192 candidates: a 128-thread CTA per row, keys in registers
-    cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sizeof(RowSmem)));
-    topk_rows_kernel<<<unsigned(rows), kRowNT, sizeof(RowSmem), s>>>(rm, blocks, tkeys, B, m, k, indices);
   } else {
     // many longer rows: one warp per row
     const int smem = kWarpRowsPerCta * (kWBins + 256) * 4;
