@@ -190,8 +190,6 @@ template <int HP, int NPW>
 __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_kernel(
     const __grid_constant__ CUtensorMap qmap, const uint16_t* __restrict__ K, const uint16_t* __restrict__ V,
     const AttnArgs a) {
-  griddep_wait();
-  griddep_launch();
   using C = Cfg<HP, NPW>;
   const int32_t* __restrict__ idx = a.idx;
   const int Lk = a.Lk, k = a.k, H = a.H;
@@ -232,6 +230,10 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
   tc_fence_after();
   const uint32_t tmem = tmem_base;
   bool dead = false;
+  // barrier set-up and the TMEM allocation above touch no global memory, so
+  // under a programmatic dependent launch they overlap the previous kernel
+  griddep_wait();
+  griddep_launch();
 
   if (warp < NPW) {
     // ------------------------------------------------------------ producers

@@ -61,23 +61,32 @@ __global__ void __launch_bounds__(256) decode_block_scores_kernel(const int32_t*
   for (int e = 0; e < VPL; ++e) q[e] = __uint_as_float(uint32_t(q_new[b * DI + lane * VPL + e]) << 16);
   const int64_t lo = 1 + int64_t(blockIdx.y) * per_cta, hi = min(nb - 1, lo + per_cta);
   const float* base = ksum_cache + b * (capacity / B) * DI;
-  for (int64_t blk = lo + warp; blk < hi; blk += 8) {
-    const float* row = base + blk * DI + lane * VPL;
-    float acc = 0.f;
-    if constexpr (VPL == 4) {
-      const float4 v = __ldg(reinterpret_cast<const float4*>(row));
-      acc = q[0] * v.x;
-      acc = __fmaf_rn(q[1], v.y, acc);
-      acc = __fmaf_rn(q[2], v.z, acc);
-      acc = __fmaf_rn(q[3], v.w, acc);
-    } else {
-      const float2 v = __ldg(reinterpret_cast<const float2*>(row));
-      acc = q[0] * v.x;
-      acc = __fmaf_rn(q[1], v.y, acc);
+  // four block rows per warp in flight before any of them is reduced
+  constexpr int U = 4;
+  for (int64_t blk0 = lo + warp; blk0 < hi; blk0 += 8 * U) {
+    float v[U][VPL];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t blk = blk0 + 8 * u;
+      const float* row = base + blk * DI + lane * VPL;
+      if constexpr (VPL == 4) {
+        const float4 x = blk < hi ? __ldg(reinterpret_cast<const float4*>(row)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        v[u][0] = x.x; v[u][1] = x.y; v[u][2] = x.z; v[u][3] = x.w;
+      } else {
+        const float2 x = blk < hi ? __ldg(reinterpret_cast<const float2*>(row)) : make_float2(0.f, 0.f);
+        v[u][0] = x.x; v[u][1] = x.y;
+      }
     }
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
-    if (lane == 0) bkeys[b * ld + blk] = score_key(acc);
+    for (int u = 0; u < U; ++u) {
+      const int64_t blk = blk0 + 8 * u;
+      float acc = q[0] * v[u][0];
+#pragma unroll
+      for (int e = 1; e < VPL; ++e) acc = __fmaf_rn(q[e], v[u][e], acc);
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
+      if (lane == 0 && blk < hi) bkeys[b * ld + blk] = score_key(acc);
+    }
   }
 }
 
