@@ -150,7 +150,10 @@ HSA_API int hsa_decode_workspace_size(const hsa_params* p, int32_t batch, int64_
  * the query at t (keys j <= t), attends, writes O [batch][H][d] bf16 and,
  * if indices_out is not NULL, the kept indices [batch][k]; then ctx_len[b]
  * += 1. A sequence with ctx_len[b] >= capacity is left untouched and its O
- * row is zero. */
+ * row is zero. The step's kernels are programmatic dependent launches: each
+ * may begin launching while the previous one runs and waits for it before
+ * touching memory, so ordering against earlier work on the stream is the
+ * usual stream order. */
 HSA_API int hsa_decode_step(const hsa_params* p, int32_t batch, int64_t capacity, int32_t* ctx_len,
                     hsa_bf16* k_idx_cache, hsa_bf16* K_cache, hsa_bf16* V_cache,
                     float* ksum_cache, const hsa_bf16* q_idx_new, const hsa_bf16* k_idx_new,

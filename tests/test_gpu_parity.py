@@ -141,6 +141,23 @@ def test_index_few_score_values_ties_exact(hsa, probs, k):
     assert np.array_equal(got, oracle.index(q, kk, 128, 16, k))
 
 
+def test_index_infinite_scores_exact(hsa):
+    # one key row whose products with every query overflow fp32 to +inf: its
+    # token score and its block's score are +inf in every row that sees it, so
+    # the top-k cannot use value-linear bins and runs on the key bits alone
+    rng = np.random.default_rng(17)
+    Lq = Lk = 3072
+    q = synth.int_bf16((Lq, 64), 17, 1)
+    q[:, 0] = synth.f32_to_bf16_bits(np.full(Lq, 2.0 ** 64, np.float32))
+    kk = synth.int_bf16((Lk, 64), 17, 2)
+    kk[:, 0] = synth.f32_to_bf16_bits(rng.integers(0, 9, Lk).astype(np.float32))
+    kk[700, 0] = synth.f32_to_bf16_bits(np.array([2.0 ** 65], np.float32))[0]
+    got = run_index(hsa, q, kk, 128, 8, 512)
+    want = oracle.index(q, kk, 128, 8, 512)
+    assert np.array_equal(got, want)
+    assert (got[1000:] == 700).any(axis=1).all()  # the +inf key is always kept once visible
+
+
 def test_index_extreme_magnitudes_exact(hsa):
     # all entries +-8: token scores reach +-8192 and block scores +-2^20
     rng = np.random.default_rng(15)
