@@ -377,20 +377,37 @@ __global__ void __launch_bounds__(kRowNT, 4) topk_rows_kernel(RowMap rm, const i
     return;
   }
   const int64_t t = rm.pos(i);
-  // the kept-block list (m <= kRowNT entries): leading entries >= 0,
-  // ascending, the query's own block last
-  const int bk = tid < m ? blocks[i * m + tid] : -1;
-  if (tid < m) S.blk[tid] = bk;
+  // stage the row's key slots first (every candidate and the unused tail);
+  // warp 0 checks the kept-block list while they land
+  {
+    const int nslot4 = (m * B) >> 2;
+    const uint4* src = reinterpret_cast<const uint4*>(tkeys + i * int64_t(m) * B);
+    for (int g = tid; g < nslot4; g += kRowNT) tc::cp_async16(tc::smem_u32(&S.keys[row_slot(g)]), src + g);
+  }
   for (int e = 0; e < kRowBPT; ++e) S.hist[tid * kRowBPT + e] = 0;
-  if (tid == 0) { S.pk[0] = m; S.red[16] = 0; }
+  if (w == 0) {
+    // leading entries >= 0 (nblk of them), ascending, the query's own block last
+    int nblk = m;
+    for (int s0 = 0; s0 < m; s0 += 32) {
+      const int s = s0 + l;
+      const int bk = s < m ? blocks[i * m + s] : -1;
+      if (s < m) S.blk[s] = bk;
+      const unsigned neg = __ballot_sync(kFull, s < m && bk < 0);
+      if (neg && nblk == m) nblk = s0 + __ffs(neg) - 1;
+    }
+    __syncwarp();
+    bool ordered = true;
+    for (int s = l; s + 1 < nblk; s += 32) ordered = ordered && S.blk[s] < S.blk[s + 1];
+    ordered = __all_sync(kFull, ordered);
+    if (l == 0) {
+      const bool ok = ordered && nblk > 0 && S.blk[nblk - 1] == int(t / B);
+      S.pk[0] = ok ? int((nblk - 1) * int64_t(B) + (t - int64_t(S.blk[nblk - 1]) * B + 1)) : -1;
+      S.red[16] = 0;
+    }
+  }
+  tc::cp_async_wait_all();
   __syncthreads();
-  if (tid < m && bk < 0) atomicMin(&S.pk[0], tid);
-  __syncthreads();
-  const int nblk = S.pk[0];
-  const bool unordered = tid + 1 < nblk && bk >= S.blk[tid + 1];
-  int n = -1;
-  if (!__syncthreads_or(unordered) && nblk > 0 && S.blk[nblk - 1] == int(t / B))
-    n = int((nblk - 1) * int64_t(B) + (t - int64_t(S.blk[nblk - 1]) * B + 1));
+  const int n = S.pk[0];
   if (n < 0) {
     for (int s = tid; s < k; s += kRowNT) out[s] = -1;
     return;
@@ -399,13 +416,6 @@ __global__ void __launch_bounds__(kRowNT, 4) topk_rows_kernel(RowMap rm, const i
   if (n <= k) {
     for (int s = tid; s < k; s += kRowNT) out[s] = s < n ? (S.blk[s >> lb] << lb) + (s & (B - 1)) : -1;
     return;
-  }
-  {
-    const int nslot4 = (m * B) >> 2;
-    const uint4* src = reinterpret_cast<const uint4*>(tkeys + i * int64_t(m) * B);
-    for (int g = tid; g < nslot4; g += kRowNT) tc::cp_async16(tc::smem_u32(&S.keys[row_slot(g)]), src + g);
-    tc::cp_async_wait_all();
-    __syncthreads();
   }
   const int p0 = tid * kRowKPT;
   const int nj = max(0, min(kRowKPT, n - p0));  // this thread's candidates: keys j < nj
@@ -446,9 +456,21 @@ __global__ void __launch_bounds__(kRowNT, 4) topk_rows_kernel(RowMap rm, const i
       cnt[e] = h4.x; cnt[e + 1] = h4.y; cnt[e + 2] = h4.z; cnt[e + 3] = h4.w;
       tot += h4.x + h4.y + h4.z + h4.w;
     }
-    int total;
-    const int above = block_exclusive_scan_rev<kRowNT>(int(tot), S.sc, &total);
-    if (uint32_t(above) < uint32_t(rem) && uint32_t(rem) <= uint32_t(above) + tot) {
+    // keys in the bins of the threads after this one: suffix sums within the
+    // warp, warp totals through shared memory (one barrier)
+    uint32_t suf = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_down_sync(kFull, suf, o);
+      if (l + o < 32) suf += y;
+    }
+    if (l == 0) S.sc[w] = int(suf);
+    __syncthreads();
+    uint32_t above = suf - tot;
+#pragma unroll
+    for (int u = 0; u < kRowNT / 32; ++u)
+      if (u > w) above += uint32_t(S.sc[u]);
+    if (above < uint32_t(rem) && uint32_t(rem) <= above + tot) {
       uint32_t a = uint32_t(above);
 #pragma unroll
       for (int e = kRowBPT - 1; e >= 0; --e) {
@@ -566,8 +588,21 @@ __global__ void __launch_bounds__(kRowNT, 4) topk_rows_kernel(RowMap rm, const i
     });
   }
   // emit in position order: slot = (#keys > T before) + min(#keys == T before, take_eq)
-  int total;
-  const int before = block_exclusive_scan<kRowNT>((__popc(gtm) << 16) | __popc(eqm), S.sc, &total);  // < 2^14 each
+  // keys before this thread's: prefix sums within the warp, warp totals
+  // through shared memory (one barrier); both counts < 2^14
+  const int mine = (__popc(gtm) << 16) | __popc(eqm);
+  int incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(kFull, incl, o);
+    if (l >= o) incl += y;
+  }
+  if (l == 31) S.sc[8 + w] = incl;
+  __syncthreads();
+  int before = incl - mine;
+#pragma unroll
+  for (int u = 0; u < kRowNT / 32; ++u)
+    if (u < w) before += S.sc[8 + u];
   int G = before >> 16, Q = before & 0xffff;
   for (uint32_t mm = gtm | eqm; mm; mm &= mm - 1u) {
     const int j = __ffs(mm) - 1;
