@@ -23,6 +23,11 @@
 // rarely after; the per-tile check is one hardware barrier reduction. P is
 // rounded to bf16 for the second MMA; accumulation is fp32.
 //
+// A barrier probe in the MMA-issuing thread costs about as much as an MMA
+// when MMAs are queued, so with two stages that thread waits on one barrier
+// per MMA group: "K tile landed and S buffer read" before S, "P written and V
+// tile landed" before PV, each counting the arrivals of both producers.
+//
 // Every mbarrier wait is bounded. Within a softmax warpgroup all four warps
 // take the same sequence of named barriers: a failed wait is folded into the
 // next barrier reduction, after which the whole warpgroup leaves together.
