@@ -107,16 +107,27 @@ __global__ void __launch_bounds__(192, 1) score_gemm_kernel(const __grid_constan
     // ------------------------------------------------------------ producer
     if (lane == 0) { prefetch_tmap(&amap); prefetch_tmap(&bmap); }
     uint32_t it = 0;
+    // a gathered tile's descriptor and query rows take two dependent global
+    // loads: they are fetched one tile ahead
+    int4 dn = make_int4(0, 0, 0, 0);
+    int rn[4] = {0, 0, 0, 0};
+    auto fetch = [&](int tt) {
+      if (tt >= total) return;
+      dn = ta.tiles[tt];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int r = lane * 4 + e;
+        rn[e] = r < dn.z ? int(ta.pairs[dn.y + r] / uint32_t(ta.m)) : 0;
+      }
+    };
+    if (GATHER) fetch(blockIdx.x);
     for (int t = blockIdx.x; t < total && !dead; t += gridDim.x) {
       int a_row0 = 0, b_row0 = 0, rows[4] = {0, 0, 0, 0};
       if (GATHER) {
-        const int4 d = ta.tiles[t];
-        b_row0 = d.x * ta.Bsz;
+        b_row0 = dn.x * ta.Bsz;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int r = lane * 4 + e;
-          rows[e] = r < d.z ? int(ta.pairs[d.y + r] / uint32_t(ta.m)) : 0;
-        }
+        for (int e = 0; e < 4; ++e) rows[e] = rn[e];
+        fetch(t + gridDim.x);
       } else {
         const int mt = t / ta.nb_tiles, nt = t % ta.nb_tiles;
         if (!block_tile_needed(ta, mt, nt, N)) continue;
