@@ -201,6 +201,14 @@ def bench_hsa(args, rank, world, device):
         step()
     torch.cuda.synchronize()
     kept = int((idx >= 0).sum().item())
+    # diagnostic: the planted needles (query i, key j with k_idx[j] = q_idx[i])
+    # whose key the selection kept
+    needles = x.get("needles", [])
+    if needles:
+        rows = idx[torch.tensor([i for i, _ in needles], device=device)].cpu().numpy()
+        needle_recall = float(np.mean([j in set(r.tolist()) for (_, j), r in zip(needles, rows)]))
+    else:
+        needle_recall = None
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     launches0 = hsa.kernel_launches()
@@ -275,6 +283,7 @@ def bench_hsa(args, rank, world, device):
         "data": "synthetic",
         "config": prefill_config(world),
         "breakdown_ms": {"hsa_index": sum(t_index) / args.steps, "hsa_sparse_attn": attn_ms},
+        "needle_recall": needle_recall,
         "roofline": {"kernel": "sparse attention", "bound": "tensor", "achieved": achieved,
                      "peak": tf, "unit": "TFLOP/s", "frac": achieved / tf,
                      "traffic": attn_traffic(w.Lq, w.L, w.d),
