@@ -441,6 +441,73 @@ def bench_reference(args, rank, world):
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+# ---------------------------------------------------------------- variants
+
+def bench_variants(device):
+    """The comparisons the pages draw, as parameter settings of the same
+    path, one JSON line each (not the headline line):
+    - the flat token-level indexer (every causal block kept, m = all blocks)
+      against the hierarchical one, at 16K where every block fits the
+      candidate limit;
+    - pure block-sparse attention: every token of the top-m blocks (k = m*B,
+      so the token stage keeps all candidates);
+    - a (B, m) sweep of the indexer at 64K with k = 2048.
+    Times are CUDA-event means of three calls after two warm-up calls."""
+    import torch
+    import hierarchical_sparse_attention_hisa_b200 as hsa
+
+    hsa.load()
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, n=3):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n
+
+    def run(name, w, x, B, m, k, attn, comment):
+        p = hsa.params(B=B, m=m, k=k, d_idx=w.d_idx, H=w.H, d=w.d)
+        q_idx, k_idx = dev_bf16(x["q_idx"], device), dev_bf16(x["k_idx"], device)
+        ws = torch.empty(max(16, hsa.hsa_index_workspace_size(p, w.Lq, w.L)), dtype=torch.uint8, device=device)
+        idx = torch.empty((w.Lq, k), dtype=torch.int32, device=device)
+        t_index = timed(lambda: hsa.hsa_index(p, w.Lq, w.L, q_idx, k_idx, idx, ws, stream))
+        res = {"variant": name, "workload": w.name, "L": w.L, "Lq": w.Lq, "B": B, "m": m, "k": k,
+               "index_ms": t_index, "note": comment}
+        if x.get("needles"):
+            rows = idx[torch.tensor([i for i, _ in x["needles"]], device=device)].cpu().numpy()
+            res["needle_recall"] = float(np.mean([j in set(r.tolist()) for (_, j), r in zip(x["needles"], rows)]))
+        del ws
+        if attn:
+            Q, K, V = (dev_bf16(x[n], device) for n in ("Q", "K", "V"))
+            O = torch.empty((w.Lq, w.H, w.d), dtype=torch.bfloat16, device=device)
+            res["attn_ms"] = timed(lambda: hsa.hsa_sparse_attn(p, w.Lq, w.L, Q, K, V, idx, O, stream))
+            res["tokens_per_s"] = w.Lq / ((t_index + res["attn_ms"]) / 1e3)
+            del Q, K, V, O
+        del idx, q_idx, k_idx
+        torch.cuda.empty_cache()
+        print(json.dumps(res), flush=True)
+
+    w16 = synth.WORKLOADS["prefill_16k"]
+    x16 = synth.prefill_inputs(w16, with_attn=False)
+    nb16 = w16.L // w16.B
+    run("hierarchical_16k", w16, x16, w16.B, w16.m, w16.k, False, "HISA indexer, m = 32 of 128 blocks")
+    run("flat_16k", w16, x16, w16.B, nb16, w16.k, False, "flat token-level indexer: every block kept")
+    del x16
+    w = PREFILL
+    x = prefill_inputs()
+    run("hierarchical_64k", w, x, w.B, w.m, w.k, True, "the headline configuration")
+    run("block_sparse_64k", w, x, w.B, w.m, w.m * w.B, True, "every token of the top-m blocks, no token stage")
+    for B, m in ((64, 16), (64, 32), (64, 64), (64, 128), (128, 16), (128, 32), (128, 64), (128, 128),
+                 (256, 32), (256, 64)):
+        run(f"sweep_B{B}_m{m}", w, x, B, m, w.k, False, "(B, m) sweep of the indexer")
+
+
 # ---------------------------------------------------------------- profiling cases
 
 def profile_case(name):
@@ -487,11 +554,17 @@ def main():
     ap.add_argument("--skip-decode", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--variants", action="store_true",
+                    help="time the flat indexer, block-sparse attention and a (B, m) sweep, then exit")
     ap.add_argument("--profile-case", choices=["attn_last8k", "index_last8k"],
                     help="run one small case for an ncu capture and exit")
     args = ap.parse_args()
     if args.profile_case:
         profile_case(args.profile_case)
+        return
+    if args.variants:
+        import torch
+        bench_variants(torch.device("cuda", 0))
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
