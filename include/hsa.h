@@ -71,8 +71,10 @@ enum {
 /* Method and layer sizes. */
 typedef struct hsa_params {
   int32_t B;     /* tokens per block, 1 <= B <= 1024                           */
-  int32_t m;     /* kept blocks per query incl. the 2 forced ones, 2 <= m <= 256 */
-  int32_t k;     /* kept tokens per query, 1 <= k <= 8192, k <= m*B            */
+  int32_t m;     /* kept blocks per query incl. the 2 forced ones, 2 <= m <= 256,
+                    m*B <= 16384 candidates                                    */
+  int32_t k;     /* kept tokens per query, 1 <= k <= 8192 (k >= m*B keeps every
+                    candidate of the kept blocks)                              */
   int32_t d_idx; /* indexer head dim: 64 or 128                                 */
   int32_t H;     /* query heads sharing one K/V head: 1 <= H <= 128             */
   int32_t d;     /* attention head dim: 64 or 128                               */
@@ -115,7 +117,8 @@ HSA_API int hsa_select_tokens(const hsa_params* p, int64_t Lq, int64_t Lk, const
 
 /* The whole indexer: block sums, block selection and token selection.
  *   q_idx [Lq][d_idx], k_idx [Lk][d_idx] bf16 -> indices [Lq][k] int32.
- * Requires 1 <= Lq <= Lk. workspace: hsa_index_workspace_size bytes. */
+ * Requires 1 <= Lq <= Lk and Lk/B <= 16384 blocks. workspace:
+ * hsa_index_workspace_size bytes. */
 HSA_API int hsa_index(const hsa_params* p, int64_t Lq, int64_t Lk, const hsa_bf16* q_idx,
               const hsa_bf16* k_idx, int32_t* indices, void* workspace, size_t workspace_bytes,
               cudaStream_t stream);
