@@ -27,3 +27,14 @@ def test_attention_traffic_scales_per_query_part_and_keeps_kv_once():
     kv = 2.0 * 65536 * 128 * 2
     t8 = bench.attn_traffic(8 * cap["queries"], 65536, 128)
     assert abs(t8 - (8 * (cap["read"] + cap["write"] - kv) + kv)) < 8.0
+
+
+def test_clock_summary_uses_samples_taken_while_timing():
+    c = bench.ClockSampler(0)
+    idle = "0, 345, 1965, 100.0, 0x0, Not Active, Not Active, Not Active, Not Active"
+    busy = "0, 1965, 1965, 900.0, 0x4, Not Active, Not Active, Not Active, Active"
+    c.lines, c.n0 = [idle, busy, busy], 1
+    s = c.summary()
+    assert s["sm_mhz"] == 1965.0 and s["samples"] == 2 and s["reasons"] == ["sw_power_cap"]
+    c.lines, c.n0 = [idle], 1  # nothing arrived during the timed work: the last sample stands in
+    assert c.summary()["samples"] == 1
