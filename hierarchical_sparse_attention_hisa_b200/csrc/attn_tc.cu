@@ -345,6 +345,9 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
           if (!wait_bar(&bars.vfull[s], (t.g / C::NS) & 1, dead)) return;
         }
         if (t.first && !wait_bar(&bars.oempty[t.ob], ((t.oq >> 1) & 1) ^ 1, dead)) return;
+        // the V rows landed by cp.async (generic proxy) are read by the MMA
+        // (async proxy): order them across proxies after the acquire above
+        fence_proxy_async_smem();
         tc_fence_after();
         const uint64_t a0 = smem_desc(smem_u32(sm + C::OFF_V + s * C::KV_BYTES), TILE * 128, 1024, kSw128);
         const uint64_t b0 = smem_desc(smem_u32(sm + C::OFF_P + pb * C::P_BYTES), 16384, 8 * C::P_ROW, C::P_SWZ);
@@ -375,6 +378,7 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
             if (!wait_bar(&bars.kfull[s], (g / C::NS) & 1, dead)) break;
             if (!wait_bar(&bars.sempty[sb], ((g >> 1) & 1) ^ 1, dead)) break;
           }
+          fence_proxy_async_smem();  // K rows landed by cp.async, read by the MMA
           tc_fence_after();
           const uint64_t kd0 = smem_desc(smem_u32(sm + C::OFF_K + s * C::KV_BYTES), 16, 1024, kSw128);
           const uint32_t klo = uint32_t(kd0), khi = uint32_t(kd0 >> 32);
