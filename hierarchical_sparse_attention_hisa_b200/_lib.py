@@ -19,7 +19,7 @@ HSA_OK, HSA_ERR_ARG, HSA_ERR_WORKSPACE, HSA_ERR_CUDA, HSA_ERR_TIMEOUT, HSA_ERR_D
 EXPORTS = (
     "hsa_status_string", "hsa_index_workspace_size", "hsa_block_sums", "hsa_select_blocks",
     "hsa_select_tokens", "hsa_index", "hsa_sparse_attn", "hsa_decode_workspace_size",
-    "hsa_decode_step", "hsa_kernel_launches", "hsa_decode_step_noalloc",
+    "hsa_decode_step", "hsa_kernel_launches", "hsa_decode_step_noalloc", "hsa_device_status",
 )
 
 
@@ -64,6 +64,7 @@ def load():
     L.hsa_decode_step.argtypes = [PP, I32, I64, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
     L.hsa_decode_step_noalloc.argtypes = [PP, I32, I64, P, P, P, P, P, P, P, P, P, P, P, P, P]
     L.hsa_kernel_launches.argtypes, L.hsa_kernel_launches.restype = [], ctypes.c_uint64
+    L.hsa_device_status.argtypes = [ctypes.c_int]
     for name in EXPORTS:
         if name not in ("hsa_status_string", "hsa_kernel_launches"):
             getattr(L, name).restype = ctypes.c_int
@@ -74,6 +75,14 @@ def load():
 def kernel_launches() -> int:
     """Kernels launched by libhsa.so in this process so far."""
     return int(load().hsa_kernel_launches())
+
+
+def hsa_device_status(reset: bool = True) -> int:
+    """HSA_OK, or HSA_ERR_TIMEOUT if a bounded device wait gave up (synchronises the device)."""
+    st = int(load().hsa_device_status(1 if reset else 0))
+    if st not in (HSA_OK, HSA_ERR_TIMEOUT):
+        raise HSAError("hsa_device_status", st)
+    return st
 
 
 def status_string(status: int) -> str:

@@ -176,6 +176,15 @@ extern "C" {
 
 uint64_t hsa_kernel_launches(void) { return hsa::g_launches.load(std::memory_order_relaxed); }
 
+int hsa_device_status(int reset) {
+  if (int e = check_device()) return e;
+  if (cudaDeviceSynchronize() != cudaSuccess) return HSA_ERR_CUDA;
+  const int a = hsa::attn_wait_flag(reset != 0);
+  const int b = hsa::score_wait_flag(reset != 0);
+  if (a < 0 || b < 0) return HSA_ERR_CUDA;
+  return a || b ? HSA_ERR_TIMEOUT : HSA_OK;
+}
+
 const char* hsa_status_string(int status) {
   switch (status) {
     case HSA_OK: return "ok";

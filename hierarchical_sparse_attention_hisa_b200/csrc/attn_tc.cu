@@ -668,4 +668,16 @@ bool launch_sparse_attn_tc_split(int batch, const void* Q, const void* Kc, const
   return launch_args(Q, Kc, Vc, a, s, pdl);
 }
 
+// Host side: whether a bounded wait of this kernel gave up on the current
+// device since the flag was last cleared (synchronous copy; -1 on a CUDA error).
+int attn_wait_flag(bool reset) {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_attn_err, sizeof v) != cudaSuccess) return -1;
+  if (reset && v) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_attn_err, &zero, sizeof zero) != cudaSuccess) return -1;
+  }
+  return v != 0;
+}
+
 }  // namespace hsa

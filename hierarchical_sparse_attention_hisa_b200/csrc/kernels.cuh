@@ -81,4 +81,9 @@ bool launch_sparse_attn_tc_split(int batch, const void* Q, const void* Kc, const
                                  float* mpart, float* lpart, cudaStream_t s, bool pdl = false);
 void launch_decode_advance(int batch, int64_t capacity, int32_t* ctx, cudaStream_t s);
 
+// Sticky per-device flags set by a bounded wait that gave up (1), read on the
+// host with a synchronous copy and optionally cleared; -1 on a CUDA error.
+int attn_wait_flag(bool reset);
+int score_wait_flag(bool reset);
+
 }  // namespace hsa

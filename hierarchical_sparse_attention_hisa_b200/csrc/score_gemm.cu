@@ -298,4 +298,16 @@ bool launch_token_score_gemm(const void* q_idx, const void* k_idx, int64_t Lq, i
   return false;
 }
 
+// Host side: whether a bounded wait of this kernel gave up on the current
+// device since the flag was last cleared (synchronous copy; -1 on a CUDA error).
+int score_wait_flag(bool reset) {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_score_err, sizeof v) != cudaSuccess) return -1;
+  if (reset && v) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_score_err, &zero, sizeof zero) != cudaSuccess) return -1;
+  }
+  return v != 0;
+}
+
 }  // namespace hsa

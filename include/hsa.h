@@ -64,7 +64,8 @@ enum {
   HSA_ERR_ARG = 1,       /* null / misaligned pointer or unsupported size  */
   HSA_ERR_WORKSPACE = 2, /* workspace missing or smaller than required      */
   HSA_ERR_CUDA = 3,      /* a CUDA launch or runtime call failed            */
-  HSA_ERR_TIMEOUT = 4,   /* a bounded device-side wait gave up              */
+  HSA_ERR_TIMEOUT = 4,   /* a bounded device-side wait gave up (reported by
+                            hsa_device_status)                              */
   HSA_ERR_DEVICE = 5     /* current device is not sm_100 (B200 class)       */
 };
 
@@ -197,6 +198,20 @@ HSA_API int hsa_decode_step_noalloc(const hsa_params* p, int32_t batch, int64_t 
  * devices, all streams) since it was loaded. A diagnostic counter for
  * benchmarks and tests; it is not synchronised with the GPU. */
 HSA_API uint64_t hsa_kernel_launches(void);
+
+/* Whether a bounded device-side wait has given up on the current device.
+ * The tensor-core kernels (block/token scoring, attention) bound every wait
+ * on an mbarrier to about two seconds of SM clock. A wait that runs out sets
+ * a sticky per-device flag; the kernel then skips the work that depended on
+ * the wait and runs to completion, so that launch's outputs are incomplete,
+ * and while the flag stays set later waits give up early. The other entry
+ * points cannot report this (they never synchronise). This call synchronises
+ * the current device (cudaDeviceSynchronize), reads the flags and returns
+ * HSA_ERR_TIMEOUT if one is set, else HSA_OK; HSA_ERR_CUDA on a CUDA error,
+ * HSA_ERR_DEVICE on a device that is not sm_100. reset != 0 clears the flags
+ * after reading them. A diagnostic for tests and benchmarks, not for the hot
+ * path. */
+HSA_API int hsa_device_status(int reset);
 
 #ifdef __cplusplus
 }

@@ -87,6 +87,14 @@ def test_bad_lengths_and_pointers_rejected(lib):
     assert lib.hsa_sparse_attn(ctypes.byref(p), 10, 20, None, None, None, None, None, None) == 1
 
 
+def test_device_status_without_a_gpu(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present: covered by test_zzz_wait_status")
+    from hierarchical_sparse_attention_hisa_b200._lib import HSA_ERR_CUDA
+    assert lib.hsa_device_status(0) == HSA_ERR_CUDA
+
+
 def test_zero_queries_is_a_no_op(lib):
     import hierarchical_sparse_attention_hisa_b200 as hsa
     p = hsa.params(B=64, m=8, k=256, d_idx=64, H=4, d=64)
