@@ -176,6 +176,51 @@ def attn_flops(idx_counts, H, d):
     return 4.0 * H * d * float(idx_counts)
 
 
+def selection_sizes(w, t):
+    """Sizes of the two selection stages for queries at positions t (array).
+
+    With nb = t // B + 1 causal blocks, nb <= m keeps every block: no block
+    score is needed and all t + 1 causal tokens are candidates. Otherwise the
+    blocks 1 .. nb - 2 are scored, and the m kept blocks are m - 1 complete
+    blocks (block 0 and the m - 2 best) plus the query's own block cut at t,
+    so (m - 1) * B + t % B + 1 tokens are candidates. min(k, candidates) keys
+    are kept. Returns (scored blocks, candidate tokens, kept keys)."""
+    t = np.asarray(t, dtype=np.int64)
+    nb = t // w.B + 1
+    pruned = nb > w.m
+    blocks = np.where(pruned, nb - 2, 0)
+    cand = np.where(pruned, (w.m - 1) * w.B + t % w.B + 1, t + 1)
+    return blocks, cand, np.minimum(cand, w.k)
+
+
+def selection_summary(w, kept):
+    """The measured number of kept (query, key) pairs beside the one the
+    selection sizes fix, and the indexer's algorithmic work against the flat
+    token-level indexer's."""
+    wm = work_model(w)
+    index_flops = wm["block_score_flops"] + wm["token_score_flops"]
+    return {"kept_pairs": int(kept), "kept_pairs_expected": wm["kept_pairs"],
+            "index_gflop": index_flops / 1e9, "flat_index_gflop": wm["flat_index_flops"] / 1e9,
+            "index_work_ratio_flat_over_hisa": wm["flat_index_flops"] / index_flops}
+
+
+def work_model(w):
+    """Algorithmic work of one prefill step of workload w (queries at
+    positions L - Lq .. L - 1): FLOPs of block scoring and token scoring (one
+    dot product of length d_idx per scored block or token), of the flat
+    token-level indexer the method replaces (every causal token scored), and
+    of the attention over the kept keys."""
+    t = np.arange(w.L - w.Lq, w.L, dtype=np.int64)
+    blocks, cand, kept = selection_sizes(w, t)
+    per = 2.0 * w.d_idx
+    kept_pairs = int(kept.sum())
+    return {"block_score_flops": per * float(blocks.sum()),
+            "token_score_flops": per * float(cand.sum()),
+            "flat_index_flops": per * float((t + 1).sum()),
+            "kept_pairs": kept_pairs,
+            "attn_flops": attn_flops(kept_pairs, w.H, w.d)}
+
+
 # ---------------------------------------------------------------- our arm
 
 def bench_hsa(args, rank, world, device):
@@ -291,6 +336,7 @@ def bench_hsa(args, rank, world, device):
         "config": prefill_config(world),
         "breakdown_ms": {"hsa_index": sum(t_index) / args.steps, "hsa_sparse_attn": attn_ms},
         "needle_recall": needle_recall,
+        "selection": selection_summary(PREFILL, kept),
         "roofline": {"kernel": "sparse attention", "bound": "tensor", "achieved": achieved,
                      "peak": tf, "unit": "TFLOP/s", "frac": achieved / tf,
                      "traffic": attn_traffic(w.Lq, w.L, w.d),
@@ -304,12 +350,13 @@ def bench_hsa(args, rank, world, device):
     return res
 
 
-def bench_decode(args, world, device):
-    """Decode: batch 32 sequences at context 131072, one query each per step."""
+def bench_decode(args, world, device, w=None):
+    """Decode: batch 32 sequences at context 131072 (or workload w's batch and
+    context), one query each per step."""
     import torch
     import hierarchical_sparse_attention_hisa_b200 as hsa
 
-    w = DECODE
+    w = DECODE if w is None else w
     steps = max(2, min(args.decode_steps, w.decode_steps))
     warm = min(args.warmup, 8)
     cap = w.decode_ctx + warm + steps + w.B
@@ -379,7 +426,9 @@ def bench_decode(args, world, device):
     per_q = (w.decode_ctx // w.B) * w.d_idx * 4 + w.m * w.B * w.d_idx * 2 + w.k * w.d * 2 * 2 \
         + 2 * w.H * w.d * 2
     gbs = per_q * w.batch / (ms / 1e3) / 1e9
-    return {"metric": "decode queries/s at 128K", "value": w.batch * world / (ms / 1e3),
+    label = "decode queries/s at 128K" if w is DECODE else \
+        f"decode queries/s ({w.name}: batch {w.batch}, context {w.decode_ctx})"
+    return {"metric": label, "value": w.batch * world / (ms / 1e3),
             "unit": "queries/s", "ms_per_step": ms, "steps_direct": half, "steps_graph": steps,
             "batch": w.batch,
             "ctx": w.decode_ctx, "timing": timing,
@@ -446,6 +495,65 @@ def bench_reference(args, rank, world):
             "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ---------------------------------------------------------------- every workload
+
+def bench_configs(args, device):
+    """Every workload timed on its own, one JSON line each (not the headline
+    line): the four prefill workloads as index + attention steps (L2 flushed
+    between steps), then the 64 decode steps at batch 1 after the 1M context.
+    Each prefill line also checks the number of kept (query, key) pairs
+    against the selection sizes the method fixes."""
+    import torch
+    import hierarchical_sparse_attention_hisa_b200 as hsa
+
+    hsa.load()
+    _, tf, _, src = peaks()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+    for name in ("tiny_prefill_2k", "prefill_16k", "prefill_64k", "prefill_1m_last8k"):
+        w = synth.WORKLOADS[name]
+        x = synth.prefill_inputs(w)
+        q_idx, k_idx = dev_bf16(x["q_idx"], device), dev_bf16(x["k_idx"], device)
+        Q, K, V = (dev_bf16(x[n], device) for n in ("Q", "K", "V"))
+        p = hsa.params(B=w.B, m=w.m, k=w.k, d_idx=w.d_idx, H=w.H, d=w.d)
+        ws = torch.empty(hsa.hsa_index_workspace_size(p, w.Lq, w.L), dtype=torch.uint8, device=device)
+        idx = torch.empty((w.Lq, w.k), dtype=torch.int32, device=device)
+        O = torch.empty((w.Lq, w.H, w.d), dtype=torch.bfloat16, device=device)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+        for s in range(args.warmup + args.steps):
+            ev = evs[s - args.warmup] if s >= args.warmup else None
+            flush.zero_()
+            if ev:
+                ev[0].record(stream)
+            hsa.hsa_index(p, w.Lq, w.L, q_idx, k_idx, idx, ws, stream)
+            if ev:
+                ev[1].record(stream)
+            hsa.hsa_sparse_attn(p, w.Lq, w.L, Q, K, V, idx, O, stream)
+            if ev:
+                ev[2].record(stream)
+        torch.cuda.synchronize()
+        t_index = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+        t_attn = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+        wm = work_model(w)
+        kept = int((idx >= 0).sum().item())
+        attn_tf = wm["attn_flops"] / (t_attn / 1e3) / 1e12
+        index_flops = wm["block_score_flops"] + wm["token_score_flops"]
+        print(json.dumps({
+            "workload": name, "L": w.L, "Lq": w.Lq, "B": w.B, "m": w.m, "k": w.k,
+            "d_idx": w.d_idx, "H": w.H, "d": w.d, "steps": args.steps, "warmup": args.warmup,
+            "value": w.Lq / ((t_index + t_attn) / 1e3), "unit": "tokens/s",
+            "ms_per_step": t_index + t_attn, "ms_index": t_index, "ms_attn": t_attn,
+            "kept_pairs": kept, "kept_pairs_expected": wm["kept_pairs"],
+            "attn_tflops": attn_tf, "attn_frac_of_bf16_peak": attn_tf / tf, "peak_source": src,
+            "index_gflop": index_flops / 1e9, "flat_index_gflop": wm["flat_index_flops"] / 1e9,
+            "index_work_ratio_flat_over_hisa": wm["flat_index_flops"] / index_flops,
+            "l2": "flushed between steps"}), flush=True)
+        del q_idx, k_idx, Q, K, V, ws, idx, O, x
+        torch.cuda.empty_cache()
+    dec = bench_decode(args, 1, device, synth.WORKLOADS["prefill_1m_last8k"])
+    print(json.dumps(dict(dec, workload="prefill_1m_last8k: decode after the 1M context")), flush=True)
 
 
 # ---------------------------------------------------------------- variants
@@ -563,6 +671,8 @@ def main():
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--variants", action="store_true",
                     help="time the flat indexer, block-sparse attention and a (B, m) sweep, then exit")
+    ap.add_argument("--configs", action="store_true",
+                    help="time every workload (2K, 16K, 64K, 1M-context chunk and its decode), then exit")
     ap.add_argument("--profile-case", choices=["attn_last8k", "index_last8k"],
                     help="run one small case for an ncu capture and exit")
     args = ap.parse_args()
@@ -572,6 +682,11 @@ def main():
     if args.variants:
         import torch
         bench_variants(torch.device("cuda", 0))
+        return
+    if args.configs:
+        import torch
+        torch.cuda.set_device(0)
+        bench_configs(args, torch.device("cuda", 0))
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
