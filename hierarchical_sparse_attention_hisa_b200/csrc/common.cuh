@@ -20,9 +20,6 @@ HSA_DEV uint32_t f32_to_bf16_rn(float f) {
   u += 0x7fffu + ((u >> 16) & 1u);
   return u >> 16;
 }
-HSA_DEV uint32_t pack_bf16x2(float lo, float hi) {
-  return f32_to_bf16_rn(lo) | (f32_to_bf16_rn(hi) << 16);
-}
 // Same rounding (nearest, ties to even) with the hardware convert.
 HSA_DEV uint32_t cvt_bf16x2(float lo, float hi) {
   uint32_t r;
