@@ -20,6 +20,7 @@ EXPORTS = (
     "hsa_status_string", "hsa_index_workspace_size", "hsa_block_sums", "hsa_select_blocks",
     "hsa_select_tokens", "hsa_index", "hsa_sparse_attn", "hsa_decode_workspace_size",
     "hsa_decode_step", "hsa_kernel_launches", "hsa_decode_step_noalloc", "hsa_device_status",
+    "hsa_prefill_host_workspace_size", "hsa_prefill_host",
 )
 
 
@@ -65,6 +66,8 @@ def load():
     L.hsa_decode_step_noalloc.argtypes = [PP, I32, I64, P, P, P, P, P, P, P, P, P, P, P, P, P]
     L.hsa_kernel_launches.argtypes, L.hsa_kernel_launches.restype = [], ctypes.c_uint64
     L.hsa_device_status.argtypes = [ctypes.c_int]
+    L.hsa_prefill_host_workspace_size.argtypes = [PP, I64, I64, ctypes.POINTER(SZ)]
+    L.hsa_prefill_host.argtypes = [PP, I64, I64, P, P, P, P, P, P, P, P, SZ, P]
     for name in EXPORTS:
         if name not in ("hsa_status_string", "hsa_kernel_launches"):
             getattr(L, name).restype = ctypes.c_int
@@ -147,6 +150,21 @@ def hsa_index(p, Lq, Lk, q_idx, k_idx, indices, workspace, stream=None):
 def hsa_sparse_attn(p, Lq, Lk, Q, K, V, indices, O, stream=None):
     _check("hsa_sparse_attn", load().hsa_sparse_attn(
         ctypes.byref(p), Lq, Lk, _p(Q), _p(K), _p(V), _p(indices), _p(O), _s(stream)))
+
+
+def hsa_prefill_host_workspace_size(p, Lq, Lk) -> int:
+    n = ctypes.c_size_t(0)
+    _check("hsa_prefill_host_workspace_size",
+           load().hsa_prefill_host_workspace_size(ctypes.byref(p), Lq, Lk, ctypes.byref(n)))
+    return n.value
+
+
+def hsa_prefill_host(p, Lq, Lk, q_idx_h, k_idx_h, Q_h, K_h, V_h, O_h, indices_h, workspace, stream=None):
+    """Index + attention with host tensors in and out (page-locked for overlap); device workspace."""
+    _check("hsa_prefill_host", load().hsa_prefill_host(
+        ctypes.byref(p), Lq, Lk, _p(q_idx_h), _p(k_idx_h), _p(Q_h), _p(K_h), _p(V_h), _p(O_h),
+        _p(indices_h), _p(workspace), workspace.numel() * workspace.element_size() if workspace is not None else 0,
+        _s(stream)))
 
 
 def hsa_decode_workspace_size(p, batch, capacity) -> int:

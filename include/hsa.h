@@ -135,6 +135,41 @@ HSA_API int hsa_sparse_attn(const hsa_params* p, int64_t Lq, int64_t Lk, const h
                     const hsa_bf16* K, const hsa_bf16* V, const int32_t* indices, hsa_bf16* O,
                     cudaStream_t stream);
 
+/* Device workspace bytes for hsa_prefill_host: device copies of its inputs
+ * and outputs plus the indexer's workspace. Checks the arguments as
+ * hsa_index and hsa_sparse_attn do (no device needed). Writes *bytes. */
+HSA_API int hsa_prefill_host_workspace_size(const hsa_params* p, int64_t Lq, int64_t Lk, size_t* bytes);
+
+/* hsa_index followed by hsa_sparse_attn for inputs and outputs in HOST
+ * memory: the end-to-end form of the path for a caller whose tensors are not
+ * on the device.
+ *   q_idx_h [Lq][d_idx], k_idx_h [Lk][d_idx], Q_h [Lq][H][d], K_h/V_h [Lk][d]:
+ *     host bf16, read;
+ *   O_h [Lq][H][d]: host bf16, written; indices_h [Lq][k]: host int32, written
+ *     unless NULL;
+ *   workspace: DEVICE memory, 256-byte aligned, of
+ *     hsa_prefill_host_workspace_size bytes.
+ * Results equal those of hsa_index + hsa_sparse_attn on the same inputs. The
+ * queries are cut into at most 8 chunks of whole 128-query tiles. Two copy
+ * streams of the library (created on a device's first call, which must not
+ * be made during stream capture, and kept until the process exits) fork from
+ * `stream` and join back into it: the indexer runs on `stream` while the Q
+ * rows come in, the attention of a chunk starts once its Q rows have landed,
+ * and a chunk's O and index rows go back while the next chunk is computed.
+ * All of it is ordered after earlier work on `stream`, and later work on
+ * `stream` runs after the last copy; the call returns once everything is
+ * enqueued (synchronise `stream` before reading O_h). The copies overlap the
+ * kernels only when the host buffers are page-locked (cudaHostAlloc,
+ * cudaHostRegister); with pageable buffers the results are the same. Calls
+ * on one device enqueue one at a time and their copies share the library's
+ * streams, in call order. Errors: those of hsa_index and hsa_sparse_attn;
+ * argument errors are returned before anything is enqueued; after a failure
+ * during enqueueing, `stream` still waits for every copy already enqueued. */
+HSA_API int hsa_prefill_host(const hsa_params* p, int64_t Lq, int64_t Lk, const hsa_bf16* q_idx_h,
+                             const hsa_bf16* k_idx_h, const hsa_bf16* Q_h, const hsa_bf16* K_h,
+                             const hsa_bf16* V_h, hsa_bf16* O_h, int32_t* indices_h,
+                             void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* Workspace bytes for hsa_decode_step. */
 HSA_API int hsa_decode_workspace_size(const hsa_params* p, int32_t batch, int64_t capacity,
                               size_t* bytes);

@@ -87,6 +87,27 @@ def test_bad_lengths_and_pointers_rejected(lib):
     assert lib.hsa_sparse_attn(ctypes.byref(p), 10, 20, None, None, None, None, None, None) == 1
 
 
+def test_prefill_host_checks_on_the_host(lib):
+    import hierarchical_sparse_attention_hisa_b200 as hsa
+    from hierarchical_sparse_attention_hisa_b200._lib import HSA_ERR_ARG, HSA_ERR_WORKSPACE
+    p = hsa.params(B=128, m=64, k=2048, d_idx=128, H=64, d=128)
+    n = hsa.hsa_prefill_host_workspace_size(p, 65536, 65536)
+    copies = 65536 * 128 * 2 * 4 + 2 * 65536 * 64 * 128 * 2 + 65536 * 2048 * 4
+    assert n >= hsa.hsa_index_workspace_size(p, 65536, 65536) + copies
+    sz = ctypes.c_size_t(0)
+    bad = hsa.params(B=128, m=64, k=2048, d_idx=128, H=0, d=128)  # an attention argument
+    assert lib.hsa_prefill_host_workspace_size(ctypes.byref(bad), 100, 200, ctypes.byref(sz)) == HSA_ERR_ARG
+    q = hsa.params(B=64, m=8, k=256, d_idx=64, H=4, d=64)
+    host = ctypes.c_void_p(0x1000)
+    # missing host buffers, then a misaligned workspace: refused before anything is enqueued
+    assert lib.hsa_prefill_host(ctypes.byref(q), 100, 200, None, None, None, None, None, None, None,
+                                None, 0, None) == HSA_ERR_ARG
+    assert lib.hsa_prefill_host(ctypes.byref(q), 100, 200, host, host, host, host, host, host, None,
+                                ctypes.c_void_p(0x1010), 1 << 30, None) == HSA_ERR_WORKSPACE
+    assert lib.hsa_prefill_host(ctypes.byref(q), 0, 200, None, None, None, None, None, None, None,
+                                None, 0, None) == 0
+
+
 def test_device_status_without_a_gpu(lib):
     import torch
     if torch.cuda.is_available():
