@@ -42,6 +42,41 @@ def test_only_declared_symbols_are_exported(lib):
     assert exported == header_functions()
 
 
+C_CALLER = r"""
+#include <string.h>
+#include "hsa.h"
+int main(void) {
+  hsa_params p = {128, 64, 2048, 128, 64, 128, 0.0f};
+  size_t n = 0;
+  if (hsa_index_workspace_size(&p, 65536, 65536, &n) != HSA_OK || n == 0) return 1;
+  if (hsa_prefill_host_workspace_size(&p, 65536, 65536, &n) != HSA_OK || n == 0) return 2;
+  if (strcmp(hsa_status_string(HSA_OK), "ok") != 0) return 3;
+  p.m = 1;
+  if (hsa_index_workspace_size(&p, 100, 200, &n) != HSA_ERR_ARG) return 4;
+  return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_links_from_c(lib, tmp_path):
+    """include/hsa.h compiles as strict C99 and a C program links libhsa.so and calls it."""
+    import shutil
+    import subprocess
+    from hierarchical_sparse_attention_hisa_b200 import lib_path
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    cuda_inc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "include")
+    src = tmp_path / "caller.c"
+    src.write_text(C_CALLER)
+    exe = tmp_path / "caller"
+    libdir = os.path.dirname(lib_path())
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I",
+                    os.path.join(ROOT, "include"), "-isystem", cuda_inc, str(src), "-L", libdir, "-lhsa",
+                    f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    assert subprocess.run([str(exe)]).returncode == 0
+
+
 def test_status_strings(lib):
     from hierarchical_sparse_attention_hisa_b200 import status_string
     assert status_string(0) == "ok"
