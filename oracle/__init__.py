@@ -18,11 +18,16 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "hsa_oracle.cpp")
 _BUILD = os.path.join(_HERE, "_build")
 _LIB = os.path.join(_BUILD, "libhsa_oracle.so")
+# A prebuilt library in place of the one built here: the mutation tests use it
+# to run the pins against copies of the oracle with a planted mistake.
+_LIB_OVERRIDE = os.environ.get("HSA_ORACLE_LIB")
 _lib = None
 
 
 def build(force: bool = False) -> str:
     """Compile the oracle with g++ (no fused multiply-add contraction)."""
+    if _LIB_OVERRIDE:
+        return _LIB_OVERRIDE
     os.makedirs(_BUILD, exist_ok=True)
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         tmp = _LIB + f".tmp{os.getpid()}"
