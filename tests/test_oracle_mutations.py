@@ -2,8 +2,9 @@
 
 Each case plants one mistake in a copy of the oracle's C++ source (a dropped
 forced block, a flipped tie rule, a wrong causal bound or query position, a
-block sum short of a row, a missing softmax scale or maximum shift, unsorted
-or zero-padded output, V swapped for K), builds it, and runs the oracle's
+block sum short of a row, a wrong range of scored blocks or block tokens, a
+missing softmax scale, maximum shift or normalisation, unsorted or
+zero-padded output, V swapped for K), builds it, and runs the oracle's
 own pin tests (tests/test_oracle.py) against it: at least one pin must
 fail. The unmodified source, built the same way, must pass them all.
 """
@@ -38,6 +39,11 @@ MUTATIONS = {
                            "    int32_t* out = indices + r * k;"),
     "padding with 0": ("static_cast<int32_t>(kept[s]) : -1;", "static_cast<int32_t>(kept[s]) : 0;"),
     "V replaced by K": ("o[c] += p * bf16_to_float(V[S[a] * d + c]);", "o[c] += p * bf16_to_float(K[S[a] * d + c]);"),
+    "block 0 among the scored": ("for (int64_t b = 1; b <= nb - 2; ++b) {", "for (int64_t b = 0; b <= nb - 2; ++b) {"),
+    "last complete block never scored": ("for (int64_t b = 1; b <= nb - 2; ++b) {",
+                                         "for (int64_t b = 1; b < nb - 2; ++b) {"),
+    "a block spills one token into the next": ("j < (b + 1) * B && j <= t; ++j)", "j <= (b + 1) * B && j <= t; ++j)"),
+    "no normalisation": ("for (int c = 0; c < d; ++c) o[c] /= l;", ""),
 }
 
 
