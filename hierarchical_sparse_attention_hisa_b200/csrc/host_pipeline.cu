@@ -13,7 +13,7 @@
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kMaxChunks = 8;
+constexpr int kMaxChunks = 16;
 constexpr size_t kAlign = 256;
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 

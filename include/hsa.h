@@ -150,7 +150,7 @@ HSA_API int hsa_prefill_host_workspace_size(const hsa_params* p, int64_t Lq, int
  *   workspace: DEVICE memory, 256-byte aligned, of
  *     hsa_prefill_host_workspace_size bytes.
  * Results equal those of hsa_index + hsa_sparse_attn on the same inputs. The
- * queries are cut into at most 8 chunks of whole 128-query tiles. Two copy
+ * queries are cut into at most 16 chunks of whole 128-query tiles. Two copy
  * streams of the library (created on a device's first call, which must not
  * be made during stream capture, and kept until the process exits) fork from
  * `stream` and join back into it: the indexer runs on `stream` while the Q
