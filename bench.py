@@ -280,6 +280,12 @@ def bench_hsa(args, rank, world, device):
     ms_step = sum(a + b for a, b in zip(t_index, t_attn)) / args.steps
     ms_step = max_over_ranks(ms_step, world, device)
     attn_ms = sum(t_attn) / args.steps
+    # rows the CPU-baseline leg checks against the oracle: evenly spaced rows
+    # and every needle row, taken from the timed steps' results
+    prow = parity_rows(w.Lq, [i for i, _ in needles])
+    prow_t = torch.from_numpy(prow).to(device)
+    parity_gpu = {"rows": prow, "idx": idx[prow_t].cpu().numpy(),
+                  "O": O[prow_t].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)}
 
     # end to end through the public API: pinned host inputs -> device, results -> host
     e2e = None
@@ -367,6 +373,7 @@ def bench_hsa(args, rank, world, device):
         "clocks": clk.summary(),
         "e2e": e2e,
         "decode": dec,
+        "_parity_gpu": parity_gpu,  # taken out before the line is printed
     }
     return res
 
@@ -471,6 +478,36 @@ def max_over_ranks(v, world, device):
 
 
 # ---------------------------------------------------------------- oracle arm
+
+def parity_rows(Lq, extra=(), n=64):
+    """n evenly spaced query rows of [0, Lq) plus the rows in `extra`, ascending."""
+    r = set(np.linspace(0, Lq - 1, n).astype(np.int64).tolist()) | {int(i) for i in extra}
+    return np.array(sorted(r), dtype=np.int64)
+
+
+def parity_summary(idx_gpu, O_gpu_bits, idx_ref, O_ref, max_abs=2e-2, mean_abs=2e-3):
+    """Rows whose indices differ at all, and the attention error of bf16 O
+    (bit patterns) against the oracle's fp64 O, with the pass/fail verdict."""
+    mism = int(np.sum(np.any(np.asarray(idx_gpu) != np.asarray(idx_ref), axis=1)))
+    got = (np.asarray(O_gpu_bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    err = np.abs(got - np.asarray(O_ref, dtype=np.float64))
+    return {"rows": int(np.asarray(idx_gpu).shape[0]), "index_rows_mismatched": mism,
+            "attn_max_abs": float(err.max()), "attn_mean_abs": float(err.mean()),
+            "tolerance": {"max_abs": max_abs, "mean_abs": mean_abs},
+            "ok": bool(mism == 0 and err.max() <= max_abs and err.mean() <= mean_abs)}
+
+
+def parity_check(gpu):
+    """The oracle on the rows bench_hsa kept from the timed steps, compared
+    with what the GPU computed for them."""
+    import oracle
+    w = PREFILL
+    x = prefill_inputs()
+    threads = oracle.default_threads()
+    idx = oracle.index(x["q_idx"], x["k_idx"], w.B, w.m, w.k, rows=gpu["rows"], threads=threads)
+    O = oracle.sparse_attn(x["Q"], x["K"], x["V"], idx, rows=gpu["rows"], threads=threads)
+    return parity_summary(gpu["idx"], gpu["O"], idx, O)
+
 
 def oracle_sample(target_s=15.0):
     """Time the oracle (index + attention) on a bounded sample of query rows
@@ -728,6 +765,7 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=device)
     res = bench_hsa(args, rank, world, device)
+    parity_gpu = res.pop("_parity_gpu", None)
     import hierarchical_sparse_attention_hisa_b200 as hsa
     # A bounded device wait that gave up leaves its launch's work undone, so
     # the line says whether every wait of the run (on every rank) completed.
@@ -737,6 +775,9 @@ def main():
         v, threads, desc = oracle_sample(target_s=float(os.environ.get("HSA_ORACLE_SECONDS", "15")))
         res["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                                "sample": desc}
+        if parity_gpu is not None:
+            # the timed steps' results against the oracle on a fixed set of rows
+            res["parity_sample"] = parity_check(parity_gpu)
     if rank == 0:
         print(json.dumps(res), flush=True)
     if world > 1:

@@ -93,3 +93,19 @@ def test_work_model_of_a_query_chunk():
     L, Lq, d = w.L, w.Lq, w.d_idx
     assert wm["flat_index_flops"] == d * (L * (L + 1) - (L - Lq) * (L - Lq + 1))
     assert wm["kept_pairs"] == Lq * w.k  # far past m*B every row keeps k
+
+
+def test_parity_rows_and_summary():
+    import numpy as np
+    rows = bench.parity_rows(65536, [5, 70000 - 10000, 0])
+    assert rows[0] == 0 and rows[-1] == 65535 and 5 in rows and 60000 in rows
+    assert np.all(np.diff(rows) > 0)
+    idx = np.arange(12, dtype=np.int32).reshape(3, 4)
+    ref_O = np.array([[[1.0, -2.0]], [[0.5, 0.25]], [[0.0, 3.0]]])
+    bits = (ref_O.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)  # exact in bf16
+    s = bench.parity_summary(idx, bits, idx.copy(), ref_O)
+    assert s["ok"] and s["index_rows_mismatched"] == 0 and s["attn_max_abs"] == 0.0
+    bad = idx.copy()
+    bad[1, 2] += 1
+    s = bench.parity_summary(bad, bits, idx, ref_O + np.array([[[0.0, 0.05]], [[0.0, 0.0]], [[0.0, 0.0]]]))
+    assert not s["ok"] and s["index_rows_mismatched"] == 1 and abs(s["attn_max_abs"] - 0.05) < 1e-12
