@@ -375,3 +375,9 @@ def test_decode_small_all_sequences(hsa):
 def test_decode_128k_two_steps_sampled(hsa):
     decode_case(hsa, B=128, m=64, k=2048, d_idx=128, H=64, d=128, ctx0=[131072] * 32,
                 capacity=131072 + 256, steps=2, seed=41, check_seqs=[0, 7, 31])
+
+
+def test_decode_after_1m_context(hsa):
+    # the decode steps of the 1M-context workload: one sequence at 1,048,576 cached tokens
+    decode_case(hsa, B=128, m=64, k=2048, d_idx=128, H=64, d=128, ctx0=[1 << 20],
+                capacity=(1 << 20) + 256, steps=2, seed=42)
