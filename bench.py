@@ -509,12 +509,13 @@ def parity_check(gpu):
     return parity_summary(gpu["idx"], gpu["O"], idx, O)
 
 
-def oracle_sample(target_s=15.0):
+def oracle_sample(target_s=15.0, w=None, x=None):
     """Time the oracle (index + attention) on a bounded sample of query rows
-    of the 64K workload; returns (tokens/s, threads, description)."""
+    of the 64K workload (or workload w with inputs x); returns (tokens/s,
+    threads, description)."""
     import oracle
-    w = PREFILL
-    x = prefill_inputs()
+    if w is None:
+        w, x = PREFILL, prefill_inputs()
     threads = oracle.default_threads()
     rows = np.linspace(0, w.Lq - 1, 8 * threads).astype(np.int64)
     t0 = time.perf_counter()
@@ -529,7 +530,7 @@ def oracle_sample(target_s=15.0):
         idx = oracle.index(x["q_idx"], x["k_idx"], w.B, w.m, w.k, rows=rows, threads=threads)
         oracle.sparse_attn(x["Q"], x["K"], x["V"], idx, rows=rows, threads=threads)
         dt = time.perf_counter() - t0
-    return n / dt, threads, f"{n} evenly spaced query rows of the 64K prefill (index + attention), {dt:.1f} s"
+    return n / dt, threads, f"{n} evenly spaced query rows of {w.name} (index + attention), {dt:.1f} s"
 
 
 def bench_reference(args, rank, world):
@@ -598,6 +599,10 @@ def bench_configs(args, device):
         kept = int((idx >= 0).sum().item())
         attn_tf = wm["attn_flops"] / (t_attn / 1e3) / 1e12
         index_flops = wm["block_score_flops"] + wm["token_score_flops"]
+        cpu = None
+        if not args.skip_cpu_baseline:  # the oracle on a bounded sample of the same workload
+            v, threads, desc = oracle_sample(target_s=float(os.environ.get("HSA_ORACLE_SECONDS", "5")), w=w, x=x)
+            cpu = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc}
         print(json.dumps({
             "workload": name, "L": w.L, "Lq": w.Lq, "B": w.B, "m": w.m, "k": w.k,
             "d_idx": w.d_idx, "H": w.H, "d": w.d, "steps": args.steps, "warmup": args.warmup,
@@ -607,7 +612,7 @@ def bench_configs(args, device):
             "attn_tflops": attn_tf, "attn_frac_of_bf16_peak": attn_tf / tf, "peak_source": src,
             "index_gflop": index_flops / 1e9, "flat_index_gflop": wm["flat_index_flops"] / 1e9,
             "index_work_ratio_flat_over_hisa": wm["flat_index_flops"] / index_flops,
-            "l2": "flushed between steps"}), flush=True)
+            "l2": "flushed between steps", "cpu_baseline": cpu}), flush=True)
         del q_idx, k_idx, Q, K, V, ws, idx, O, x
         torch.cuda.empty_cache()
     dec = bench_decode(args, 1, device, synth.WORKLOADS["prefill_1m_last8k"])
