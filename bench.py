@@ -774,8 +774,13 @@ def main():
     import hierarchical_sparse_attention_hisa_b200 as hsa
     # A bounded device wait that gave up leaves its launch's work undone, so
     # the line says whether every wait of the run (on every rank) completed.
-    gave_up = max_over_ranks(float(hsa.hsa_device_status(reset=True) != 0), world, device)
-    res["device_waits"] = "a bounded wait gave up: outputs incomplete" if gave_up else "all completed"
+    try:
+        status = float(hsa.hsa_device_status(reset=True) != 0)
+    except hsa.HSAError as ex:  # the check itself failed: say so, keep the line
+        status, res["device_waits_error"] = -1.0, str(ex)
+    gave_up = max_over_ranks(status, world, device)
+    res["device_waits"] = ("a bounded wait gave up: outputs incomplete" if gave_up > 0 else
+                           "all completed" if gave_up == 0 else "not checked")
     if rank == 0 and world == 1 and not args.skip_cpu_baseline:
         v, threads, desc = oracle_sample(target_s=float(os.environ.get("HSA_ORACLE_SECONDS", "15")))
         res["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
