@@ -27,7 +27,7 @@ constexpr int64_t kMaxCandidates = 16384;
 int check_device() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return HSA_ERR_CUDA;
-  static int cached_dev = -1, cached_ok = 0;
+  thread_local int cached_dev = -1, cached_ok = 0;  // per host thread: no shared mutable state
   if (dev != cached_dev) {
     int major = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)

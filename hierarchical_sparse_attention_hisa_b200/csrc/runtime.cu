@@ -40,7 +40,7 @@ bool make_tmap_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols
 int num_sms() {
   int dev = 0, v = 148;
   cudaGetDevice(&dev);
-  static int cached_dev = -1, cached = 148;
+  thread_local int cached_dev = -1, cached = 148;  // per host thread: no shared mutable state
   if (dev != cached_dev) {
     cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
     cached = v;
