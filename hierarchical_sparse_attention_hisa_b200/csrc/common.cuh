@@ -34,7 +34,6 @@ HSA_DEV uint32_t score_key(float f) {
   if ((u << 1) == 0u) u = 0u;
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
-// The score a key stands for (inverse of score_key; -0 comes back as +0).
 // Programmatic dependent launch. A kernel launched with the attribute may
 // start while the previous kernel of its stream is still running; it calls
 // griddep_wait() before touching any memory that kernel reads or writes (the
@@ -44,6 +43,7 @@ HSA_DEV uint32_t score_key(float f) {
 HSA_DEV void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 HSA_DEV void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// The score a key stands for (inverse of score_key; -0 comes back as +0).
 HSA_DEV float key_score(uint32_t u) { return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u); }
 
 // Which absolute position a query row has, and where its sequence lives.

@@ -220,7 +220,11 @@ HSA_API int hsa_decode_step(const hsa_params* p, int32_t batch, int64_t capacity
  * (cudaGetSymbolAddress, with that device current); make that first call
  * before capturing the stream into a CUDA graph. Every call on a device
  * shares the one array and leaves its contents behind: two calls whose work
- * overlaps on the GPU (different streams without ordering) race on it. */
+ * overlaps on the GPU (different streams without ordering) race on it.
+ * The looked-up address is kept for the life of the process: after
+ * cudaDeviceReset on a device, the library's per-device state for that device
+ * (this address, and the copy streams of hsa_prefill_host) is stale, so do not
+ * call into the library on a device that has been reset. */
 HSA_API int hsa_decode_step_noalloc(const hsa_params* p, int32_t batch, int64_t capacity,
                                     int32_t* ctx_len, hsa_bf16* k_idx_cache, hsa_bf16* K_cache,
                                     hsa_bf16* V_cache, float* ksum_cache,
