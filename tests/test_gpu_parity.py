@@ -199,6 +199,23 @@ def test_index_long_context_chunk_all_rows(hsa):
     assert bad.size == 0, f"{bad.size} rows differ, first {bad[:8].tolist()}"
 
 
+@pytest.mark.parametrize("Lq,Lk,B,m,k,seed", [
+    (16384, 16384, 128, 128, 2048, 50),  # the flat token-level indexer at 16K: every causal block kept
+    (1000, 12000, 128, 80, 1000, 52),    # 10,240 candidates, many rows: one warp per row
+    (400, 20000, 64, 200, 3000, 53),     # 12,800 candidates at B = 64
+    (200, 40000, 64, 256, 2048, 51),     # 16,384 candidates, few rows: a 1024-thread CTA per row
+    (100, 30000, 128, 100, 4096, 54),    # 12,800 candidates, few rows, k above the block count * 32
+])
+def test_index_long_candidate_rows_bit_exact(hsa, Lq, Lk, B, m, k, seed):
+    # rows of more than 8192 candidates (m*B > 8192) leave the shared-memory
+    # row kernel of the top-k for the longer-row kernels
+    q, kk = synth.int_bf16((Lq, 128), seed, 1), synth.int_bf16((Lk, 128), seed, 2)
+    got = run_index(hsa, q, kk, B, m, k)
+    want = oracle.index(q, kk, B, m, k)
+    bad = np.flatnonzero(np.any(got != want, axis=1))
+    assert bad.size == 0, f"{bad.size} rows differ, first {bad[:8].tolist()}"
+
+
 # ------------------------------------------------------------------ attention
 
 def test_attention_tiny_prefill_all_rows(hsa):
@@ -233,6 +250,35 @@ def test_attention_shapes(hsa, H, d, k):
     got = run_attn(hsa, Q, K, V, idx)
     ref = oracle.sparse_attn(Q, K, V, idx)
     assert_attn_close(got, ref, f"H={H} d={d} k={k}")
+
+
+@pytest.mark.parametrize("k", [4096, 8192])
+def test_attention_long_index_rows(hsa, k):
+    # k above 2048 (up to the 8192 the API accepts): 32 or 64 tiles per query,
+    # ragged and empty rows among them
+    Lq, Lk, H, d = 40, 12000, 64, 128
+    rng = np.random.default_rng(k)
+    Q, K, V = (synth.normal_bf16(s, 26, i) for i, s in enumerate([(Lq, H, d), (Lk, d), (Lk, d)]))
+    idx = np.full((Lq, k), -1, dtype=np.int32)
+    for i in range(Lq):
+        n = k if i % 3 == 0 else int(rng.integers(0, k + 1))
+        idx[i, :n] = np.sort(rng.choice(Lk, size=n, replace=False))
+    got = run_attn(hsa, Q, K, V, idx)
+    assert_attn_close(got, oracle.sparse_attn(Q, K, V, idx), f"k={k}")
+
+
+def test_attention_pure_block_sparse_64k_sampled(hsa):
+    # the pure block-sparse setting of the 64K workload: k = m*B keeps every
+    # candidate of the top-m blocks (8192 keys per query)
+    w = synth.WORKLOADS["prefill_64k"]
+    x = synth.prefill_inputs(w)
+    k = w.m * w.B
+    idx = run_index(hsa, x["q_idx"], x["k_idx"], w.B, w.m, k)
+    rows = sample_rows(w.Lq, 256, 27, always=[0, w.B * w.m, w.Lq - 1])
+    assert np.array_equal(idx[rows], oracle.index(x["q_idx"], x["k_idx"], w.B, w.m, k, rows=rows))
+    got = run_attn(hsa, x["Q"], x["K"], x["V"], idx)
+    ref = oracle.sparse_attn(x["Q"], x["K"], x["V"], idx[rows], rows=rows)
+    print("64k block-sparse max/mean abs err", assert_attn_close(got[rows], ref, "64k k=8192"))
 
 
 def test_attention_large_logits_stable(hsa):
@@ -372,9 +418,13 @@ def test_decode_small_all_sequences(hsa):
                 capacity=1024, steps=70, seed=40)
 
 
-def test_decode_128k_two_steps_sampled(hsa):
-    decode_case(hsa, B=128, m=64, k=2048, d_idx=128, H=64, d=128, ctx0=[131072] * 32,
-                capacity=131072 + 256, steps=2, seed=41, check_seqs=[0, 7, 31])
+def test_decode_128k_all_sequences(hsa):
+    # the 128K decode workload's shape, every sequence checked: the contexts
+    # start one token short of 1024 full blocks, so step 0 completes block
+    # 1023 of every sequence (its block sum is written and then compared) and
+    # step 1 scores it as a candidate block
+    decode_case(hsa, B=128, m=64, k=2048, d_idx=128, H=64, d=128, ctx0=[131071] * 32,
+                capacity=131072 + 256, steps=2, seed=41)
 
 
 def test_decode_after_1m_context(hsa):
