@@ -287,6 +287,21 @@ def bench_hsa(args, rank, world, device):
     parity_gpu = {"rows": prow, "idx": idx[prow_t].cpu().numpy(),
                   "O": O[prow_t].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)}
 
+    # the indexer's two stages on their own, for the workload's configs entry
+    t_block, t_token = time_index_stages(args, w, p, q_idx, k_idx, ws, idx, flush, stream)
+    wmh = work_model(w)
+    hbm_, tf_, _, src_ = peaks()
+    attn_tf_ = wmh["attn_flops"] / (attn_ms / 1e3) / 1e12
+    configs_headline = {
+        "L": w.L, "Lq": w.Lq, "B": w.B, "m": w.m, "k": w.k, "d_idx": w.d_idx, "H": w.H, "d": w.d,
+        "ms_index": sum(t_index) / args.steps, "ms_attn": attn_ms,
+        "ms_index_block_stage": t_block, "ms_index_token_stage": t_token,
+        "kept_pairs": kept, "kept_pairs_expected": wmh["kept_pairs"],
+        "roofline": {"attention": {"bound": "tensor", "achieved": attn_tf_, "peak": tf_, "unit": "TFLOP/s",
+                                   "frac": attn_tf_ / tf_, "peak_source": f"{src_} bf16 burst"},
+                     **index_rooflines(w, t_block, t_token)},
+        "l2": "flushed between steps", "note": "the headline workload: the line's own figures"}
+
     # end to end through the public API: pinned host inputs -> device, results -> host
     e2e = None
     if not args.skip_e2e:
@@ -374,6 +389,7 @@ def bench_hsa(args, rank, world, device):
         "e2e": e2e,
         "decode": dec,
         "_parity_gpu": parity_gpu,  # taken out before the line is printed
+        "configs_headline": configs_headline,  # becomes the headline's entry of `configs`
     }
     return res
 
@@ -558,65 +574,184 @@ def bench_reference(args, rank, world):
 
 # ---------------------------------------------------------------- every workload
 
-def bench_configs(args, device):
-    """Every workload timed on its own, one JSON line each (not the headline
-    line): the four prefill workloads as index + attention steps (L2 flushed
-    between steps), then the 64 decode steps at batch 1 after the 1M context.
-    Each prefill line also checks the number of kept (query, key) pairs
-    against the selection sizes the method fixes."""
+def time_index_stages(args, w, p, q_idx, k_idx, ws, idx, flush, stream):
+    """The indexer's two selection stages timed on their own through the
+    stage entry points hsa_index chains (L2 flushed before each pass):
+    block stage = block sums + block scoring + top-m, token stage = token
+    scoring + top-k. Returns their mean times in ms."""
     import torch
     import hierarchical_sparse_attention_hisa_b200 as hsa
 
-    hsa.load()
-    _, tf, _, src = peaks()
+    device = q_idx.device
+    ksum = torch.empty((max(w.L // w.B, 1), w.d_idx), dtype=torch.float32, device=device)
+    blocks = torch.empty((w.Lq, w.m), dtype=torch.int32, device=device)
+    steps = max(1, args.steps)
+    sev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for s in range(args.warmup + steps):
+        ev = sev[s - args.warmup] if s >= args.warmup else None
+        flush.zero_()
+        if ev:
+            ev[0].record(stream)
+        hsa.hsa_block_sums(p, w.L, k_idx, ksum, stream)
+        hsa.hsa_select_blocks(p, w.Lq, w.L, q_idx, ksum, blocks, ws, stream)
+        if ev:
+            ev[1].record(stream)
+        hsa.hsa_select_tokens(p, w.Lq, w.L, q_idx, k_idx, blocks, idx, ws, stream)
+        if ev:
+            ev[2].record(stream)
+    torch.cuda.synchronize()
+    return (statistics.mean(e[0].elapsed_time(e[1]) for e in sev),
+            statistics.mean(e[1].elapsed_time(e[2]) for e in sev))
+
+
+def index_rooflines(w, t_block, t_token):
+    """Roofline entries of the indexer's two stages (see time_index_stages)."""
+    hbm, tf, _, src = peaks()
+    wm = work_model(w)
+    block_tf = 3 * wm["block_score_flops"] / (t_block / 1e3) / 1e12
+    # token scoring's algorithmic bytes: the d_idx bf16 values of every
+    # candidate key each query scores (one dot product per candidate, so the
+    # same count as its FLOPs); reuse through L2 can carry this past HBM peak
+    token_gbs = wm["token_score_flops"] / (t_token / 1e3) / 1e9
+    return {
+        "block_stage": {"bound": "tensor", "achieved": block_tf, "peak": tf, "unit": "TFLOP/s",
+                        "frac": block_tf / tf, "peak_source": f"{src} bf16 burst",
+                        "note": "three bf16 planes of the fp32 block sums, so 3x the block-score FLOPs; "
+                                "the stage time includes the block sums and the top-m"},
+        "token_stage": {"bound": "hbm", "achieved": token_gbs, "peak": hbm, "unit": "GB/s",
+                        "frac": token_gbs / hbm, "peak_source": f"{src} copy",
+                        "note": "effective: candidate keys' bytes / stage time (MMA reuse through L2 "
+                                "can carry it past HBM peak); the stage time includes the top-k"}}
+
+
+def time_prefill(args, w, x, device, flush, stream):
+    """One prefill workload timed as index + attention steps (L2 flushed
+    between steps), plus the index's two selection stages timed on their own
+    (block stage: block sums + block scoring + top-m; token stage: token
+    scoring + top-k, through the stage entry points hsa_index chains).
+    Returns the workload's entry of the bench line's `configs` object."""
+    import torch
+    import hierarchical_sparse_attention_hisa_b200 as hsa
+
+    hbm, tf, _, src = peaks()
+    q_idx, k_idx = dev_bf16(x["q_idx"], device), dev_bf16(x["k_idx"], device)
+    Q, K, V = (dev_bf16(x[n], device) for n in ("Q", "K", "V"))
+    p = hsa.params(B=w.B, m=w.m, k=w.k, d_idx=w.d_idx, H=w.H, d=w.d)
+    ws = torch.empty(hsa.hsa_index_workspace_size(p, w.Lq, w.L), dtype=torch.uint8, device=device)
+    idx = torch.empty((w.Lq, w.k), dtype=torch.int32, device=device)
+    O = torch.empty((w.Lq, w.H, w.d), dtype=torch.bfloat16, device=device)
+    steps = max(1, args.steps)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for s in range(args.warmup + steps):
+        ev = evs[s - args.warmup] if s >= args.warmup else None
+        flush.zero_()
+        if ev:
+            ev[0].record(stream)
+        hsa.hsa_index(p, w.Lq, w.L, q_idx, k_idx, idx, ws, stream)
+        if ev:
+            ev[1].record(stream)
+        hsa.hsa_sparse_attn(p, w.Lq, w.L, Q, K, V, idx, O, stream)
+        if ev:
+            ev[2].record(stream)
+    torch.cuda.synchronize()
+    t_index = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    t_attn = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    wm = work_model(w)
+    kept = int((idx >= 0).sum().item())
+    attn_tf = wm["attn_flops"] / (t_attn / 1e3) / 1e12
+    index_flops = wm["block_score_flops"] + wm["token_score_flops"]
+    t_block, t_token = time_index_stages(args, w, p, q_idx, k_idx, ws, idx, flush, stream)
+    res = {
+        "L": w.L, "Lq": w.Lq, "B": w.B, "m": w.m, "k": w.k, "d_idx": w.d_idx, "H": w.H, "d": w.d,
+        "value": w.Lq / ((t_index + t_attn) / 1e3), "unit": "tokens/s",
+        "ms_per_step": t_index + t_attn, "ms_index": t_index, "ms_attn": t_attn,
+        "ms_index_block_stage": t_block, "ms_index_token_stage": t_token,
+        "kept_pairs": kept, "kept_pairs_expected": wm["kept_pairs"],
+        "roofline": {
+            "attention": {"bound": "tensor", "achieved": attn_tf, "peak": tf, "unit": "TFLOP/s",
+                          "frac": attn_tf / tf, "peak_source": f"{src} bf16 burst"},
+            **index_rooflines(w, t_block, t_token)},
+        "index_gflop": index_flops / 1e9, "flat_index_gflop": wm["flat_index_flops"] / 1e9,
+        "index_work_ratio_flat_over_hisa": wm["flat_index_flops"] / index_flops,
+        "l2": "flushed between steps"}
+    del q_idx, k_idx, Q, K, V, ws, idx, O
+    torch.cuda.empty_cache()
+    return res
+
+
+def bench_configs(args, device, headline=None):
+    """Every workload but the headline one, timed on its own: the prefill
+    workloads (2K, 16K, the last 8192 queries of the 1M context) as index +
+    attention steps, then the 64 batch-1 decode steps after the 1M context.
+    Each entry also checks its number of kept (query, key) pairs against the
+    selection sizes the method fixes, and carries a bounded oracle sample of
+    the same workload (host cores). Returns {workload: entry}."""
+    import torch
+
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream()
+    out = {}
     for name in ("tiny_prefill_2k", "prefill_16k", "prefill_64k", "prefill_1m_last8k"):
+        if name == PREFILL.name and headline is not None:
+            out[name] = headline
+            continue
         w = synth.WORKLOADS[name]
         x = synth.prefill_inputs(w)
-        q_idx, k_idx = dev_bf16(x["q_idx"], device), dev_bf16(x["k_idx"], device)
-        Q, K, V = (dev_bf16(x[n], device) for n in ("Q", "K", "V"))
-        p = hsa.params(B=w.B, m=w.m, k=w.k, d_idx=w.d_idx, H=w.H, d=w.d)
-        ws = torch.empty(hsa.hsa_index_workspace_size(p, w.Lq, w.L), dtype=torch.uint8, device=device)
-        idx = torch.empty((w.Lq, w.k), dtype=torch.int32, device=device)
-        O = torch.empty((w.Lq, w.H, w.d), dtype=torch.bfloat16, device=device)
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-        for s in range(args.warmup + args.steps):
-            ev = evs[s - args.warmup] if s >= args.warmup else None
-            flush.zero_()
-            if ev:
-                ev[0].record(stream)
-            hsa.hsa_index(p, w.Lq, w.L, q_idx, k_idx, idx, ws, stream)
-            if ev:
-                ev[1].record(stream)
-            hsa.hsa_sparse_attn(p, w.Lq, w.L, Q, K, V, idx, O, stream)
-            if ev:
-                ev[2].record(stream)
-        torch.cuda.synchronize()
-        t_index = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-        t_attn = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-        wm = work_model(w)
-        kept = int((idx >= 0).sum().item())
-        attn_tf = wm["attn_flops"] / (t_attn / 1e3) / 1e12
-        index_flops = wm["block_score_flops"] + wm["token_score_flops"]
-        cpu = None
+        res = time_prefill(args, w, x, device, flush, stream)
         if not args.skip_cpu_baseline:  # the oracle on a bounded sample of the same workload
-            v, threads, desc = oracle_sample(target_s=float(os.environ.get("HSA_ORACLE_SECONDS", "5")), w=w, x=x)
-            cpu = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc}
-        print(json.dumps({
-            "workload": name, "L": w.L, "Lq": w.Lq, "B": w.B, "m": w.m, "k": w.k,
-            "d_idx": w.d_idx, "H": w.H, "d": w.d, "steps": args.steps, "warmup": args.warmup,
-            "value": w.Lq / ((t_index + t_attn) / 1e3), "unit": "tokens/s",
-            "ms_per_step": t_index + t_attn, "ms_index": t_index, "ms_attn": t_attn,
-            "kept_pairs": kept, "kept_pairs_expected": wm["kept_pairs"],
-            "attn_tflops": attn_tf, "attn_frac_of_bf16_peak": attn_tf / tf, "peak_source": src,
-            "index_gflop": index_flops / 1e9, "flat_index_gflop": wm["flat_index_flops"] / 1e9,
-            "index_work_ratio_flat_over_hisa": wm["flat_index_flops"] / index_flops,
-            "l2": "flushed between steps", "cpu_baseline": cpu}), flush=True)
-        del q_idx, k_idx, Q, K, V, ws, idx, O, x
-        torch.cuda.empty_cache()
-    dec = bench_decode(args, 1, device, synth.WORKLOADS["prefill_1m_last8k"])
-    print(json.dumps(dict(dec, workload="prefill_1m_last8k: decode after the 1M context")), flush=True)
+            v, threads, desc = oracle_sample(target_s=float(os.environ.get("HSA_ORACLE_SECONDS_CFG", "5")), w=w, x=x)
+            res["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                                   "sample": desc}
+        out[name] = res
+        del x
+    del flush
+    torch.cuda.empty_cache()
+    out["prefill_1m_last8k_decode"] = bench_decode(args, 1, device, synth.WORKLOADS["prefill_1m_last8k"])
+    out["flat_indexer_64k"] = bench_flat_indexer(args, device, headline)
+    return out
+
+
+def bench_flat_indexer(args, device, headline=None):
+    """The token-level indexer the method replaces (the pages' comparison):
+    the same library with every causal block kept (m = all 512 blocks of the
+    64K workload), so every causal token of a query is scored and the top-k
+    taken over all of them. Timed like the hierarchical indexer (L2 flushed
+    between calls) and reported beside it."""
+    import torch
+    import hierarchical_sparse_attention_hisa_b200 as hsa
+
+    w = PREFILL
+    x = synth.prefill_inputs(w, with_attn=False)
+    q_idx, k_idx = dev_bf16(x["q_idx"], device), dev_bf16(x["k_idx"], device)
+    m_flat = w.L // w.B
+    p = hsa.params(B=w.B, m=m_flat, k=w.k, d_idx=w.d_idx, H=w.H, d=w.d)
+    ws = torch.empty(hsa.hsa_index_workspace_size(p, w.Lq, w.L), dtype=torch.uint8, device=device)
+    idx = torch.empty((w.Lq, w.k), dtype=torch.int32, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+    steps = max(1, min(args.steps, 3))
+    ts = []
+    for s in range(args.warmup + steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        hsa.hsa_index(p, w.Lq, w.L, q_idx, k_idx, idx, ws, stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if s >= args.warmup:
+            ts.append(a.elapsed_time(b))
+    ms = statistics.mean(ts)
+    wm = work_model(w)
+    res = {"m": m_flat, "ms_index": ms, "index_gflop": wm["flat_index_flops"] / 1e9,
+           "workspace_bytes": int(ws.numel())}
+    if headline is not None and headline.get("ms_index"):
+        res["ms_index_hisa"] = headline["ms_index"]
+        res["speedup_hisa_over_flat"] = ms / headline["ms_index"]
+    res["note"] = ("context, not a target: the HISA page reports up to 3.75x over the DSA indexer at 64K "
+                   "(hardware not stated)")
+    del ws, idx, q_idx, k_idx, flush
+    torch.cuda.empty_cache()
+    return res
 
 
 # ---------------------------------------------------------------- variants
@@ -690,10 +825,19 @@ def bench_variants(device):
 
 def profile_case(name):
     """Small cases for ncu captures: the last 8192 queries of the 64K workload
-    (inputs larger than L2), run three times untimed and once timed."""
+    (inputs larger than L2), run three times untimed and once timed; or
+    decode_128k: 12 steps of the batch-32 decode at context 131072 (the
+    caches, about 3.3 GB, far larger than L2)."""
     import torch
     import hierarchical_sparse_attention_hisa_b200 as hsa
     hsa.load()
+    if name == "decode_128k":
+        class A:  # the decode bench's arguments
+            decode_steps, warmup = 4, 8
+        torch.cuda.set_device(0)
+        dec = bench_decode(A(), 1, torch.device("cuda", 0))
+        print(json.dumps({"profile_case": name, "ms_per_step": dec["ms_per_step"]}))
+        return
     w = PREFILL
     lq = 8192
     x = synth.prefill_inputs(w, with_attn=(name == "attn_last8k"))
@@ -732,11 +876,13 @@ def main():
     ap.add_argument("--skip-decode", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--skip-configs", action="store_true",
+                    help="leave out the other workloads' entries (configs) of the line")
     ap.add_argument("--variants", action="store_true",
                     help="time the flat indexer, block-sparse attention and a (B, m) sweep, then exit")
     ap.add_argument("--configs", action="store_true",
                     help="time every workload (2K, 16K, 64K, 1M-context chunk and its decode), then exit")
-    ap.add_argument("--profile-case", choices=["attn_last8k", "index_last8k"],
+    ap.add_argument("--profile-case", choices=["attn_last8k", "index_last8k", "decode_128k"],
                     help="run one small case for an ncu capture and exit")
     args = ap.parse_args()
     if args.profile_case:
@@ -749,7 +895,10 @@ def main():
     if args.configs:
         import torch
         torch.cuda.set_device(0)
-        bench_configs(args, torch.device("cuda", 0))
+        import hierarchical_sparse_attention_hisa_b200 as hsa
+        hsa.load()
+        for name, entry in bench_configs(args, torch.device("cuda", 0)).items():
+            print(json.dumps(dict(entry, workload=name)), flush=True)
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -791,6 +940,13 @@ def main():
                 res["parity_sample"] = parity_check(parity_gpu)
             except Exception as ex:  # the line is still printed, saying why the check is missing
                 res["parity_sample"] = {"error": f"{type(ex).__name__}: {ex}"}
+    if world == 1 and not args.skip_configs:
+        # the other workloads, each on its own (one GPU only: the headline
+        # numbers above are what the replicas of a multi-GPU run measure)
+        head = {k: res[k] for k in ("value", "unit", "ms_per_step")}
+        head.update(res.get("configs_headline", {}))
+        res["configs"] = bench_configs(args, device, headline=head)
+    res.pop("configs_headline", None)
     if rank == 0:
         print(json.dumps(res), flush=True)
     if world > 1:

@@ -14,7 +14,8 @@ see include/hsa.h); this package marshals torch tensors into it.
 from __future__ import annotations
 
 from ._lib import (EXPORTS, HSAError, hsa_block_sums, hsa_decode_step,  # noqa: F401
-                   hsa_decode_step_noalloc, hsa_device_status, hsa_prefill_host,
+                   hsa_debug_inject_lost_arrival, hsa_decode_step_noalloc, hsa_device_status,
+                   hsa_prefill_host,
                    hsa_prefill_host_workspace_size,
                    hsa_decode_workspace_size, hsa_index, hsa_index_workspace_size, hsa_params,
                    hsa_select_blocks, hsa_select_tokens, hsa_sparse_attn, kernel_launches, lib_path, load,

@@ -20,7 +20,7 @@ EXPORTS = (
     "hsa_status_string", "hsa_index_workspace_size", "hsa_block_sums", "hsa_select_blocks",
     "hsa_select_tokens", "hsa_index", "hsa_sparse_attn", "hsa_decode_workspace_size",
     "hsa_decode_step", "hsa_kernel_launches", "hsa_decode_step_noalloc", "hsa_device_status",
-    "hsa_prefill_host_workspace_size", "hsa_prefill_host",
+    "hsa_prefill_host_workspace_size", "hsa_prefill_host", "hsa_debug_inject_lost_arrival",
 )
 
 
@@ -66,6 +66,7 @@ def load():
     L.hsa_decode_step_noalloc.argtypes = [PP, I32, I64, P, P, P, P, P, P, P, P, P, P, P, P, P]
     L.hsa_kernel_launches.argtypes, L.hsa_kernel_launches.restype = [], ctypes.c_uint64
     L.hsa_device_status.argtypes = [ctypes.c_int]
+    L.hsa_debug_inject_lost_arrival.argtypes = [ctypes.c_int]
     L.hsa_prefill_host_workspace_size.argtypes = [PP, I64, I64, ctypes.POINTER(SZ)]
     L.hsa_prefill_host.argtypes = [PP, I64, I64, P, P, P, P, P, P, P, P, SZ, P]
     for name in EXPORTS:
@@ -86,6 +87,11 @@ def hsa_device_status(reset: bool = True) -> int:
     if st not in (HSA_OK, HSA_ERR_TIMEOUT):
         raise HSAError("hsa_device_status", st)
     return st
+
+
+def hsa_debug_inject_lost_arrival(on: bool) -> None:
+    """Test hook: short bounded waits and one lost producer hand-off per tensor-core kernel."""
+    _check("hsa_debug_inject_lost_arrival", int(load().hsa_debug_inject_lost_arrival(1 if on else 0)))
 
 
 def status_string(status: int) -> str:

@@ -21,8 +21,15 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Candidates a selection stage keeps in shared memory per query.
-constexpr int64_t kMaxCandidates = 16384;
+// Blocks of a sequence the block stage scores per query.
+constexpr int64_t kMaxBlocks = 16384;
+// Token candidates per query (kept blocks x B): the tensor-core token scoring
+// with its key-stream top-k takes up to kMaxCandidates, the CUDA-core token
+// scoring (block sizes the MMA cannot take) stages them in shared memory and
+// takes up to kMaxCandidatesSmem.
+constexpr int64_t kMaxCandidates = 65536;
+constexpr int64_t kMaxCandidatesSmem = 16384;
+constexpr int kMaxM = 512;  // kept blocks per query
 
 int check_device() {
   int dev = 0;
@@ -41,10 +48,11 @@ int check_device() {
 int check_index_params(const hsa_params* p) {
   if (!p) return HSA_ERR_ARG;
   if (p->B < 1 || p->B > 1024) return HSA_ERR_ARG;
-  if (p->m < 2 || p->m > 256) return HSA_ERR_ARG;
+  if (p->m < 2 || p->m > kMaxM) return HSA_ERR_ARG;
   if (p->k < 1 || p->k > 8192) return HSA_ERR_ARG;
   if (p->d_idx != 64 && p->d_idx != 128) return HSA_ERR_ARG;
-  if (int64_t(p->m) * p->B > kMaxCandidates) return HSA_ERR_ARG;
+  const bool mma_tokens = p->B == 64 || p->B == 128 || p->B == 256;
+  if (int64_t(p->m) * p->B > (mma_tokens ? kMaxCandidates : kMaxCandidatesSmem)) return HSA_ERR_ARG;
   return HSA_OK;
 }
 
@@ -64,7 +72,7 @@ float softmax_scale(const hsa_params* p) {
 int check_lengths(const hsa_params* p, int64_t Lq, int64_t Lk) {
   if (Lq < 0 || Lk < 1 || Lq > Lk || Lq > (int64_t(1) << 31) - 1) return HSA_ERR_ARG;
   if (Lk > (int64_t(1) << 31) - 1) return HSA_ERR_ARG;
-  if (Lk / p->B > kMaxCandidates) return HSA_ERR_ARG;
+  if (Lk / p->B > kMaxBlocks) return HSA_ERR_ARG;
   return HSA_OK;
 }
 
@@ -120,7 +128,7 @@ bool block_gemm_ok(const hsa_params* p, int64_t Lq, int64_t Lk) {
   return Lq >= 128 && 3 * (Lk / p->B) >= 64;
 }
 bool token_gemm_ok(const hsa_params* p, int64_t Lq, int64_t Lk) {
-  return (p->B == 64 || p->B == 128) && Lk >= p->B && Lq * int64_t(p->m) < (int64_t(1) << 32);
+  return (p->B == 64 || p->B == 128 || p->B == 256) && Lk >= p->B && Lq * int64_t(p->m) < (int64_t(1) << 32);
 }
 
 // Kept blocks for rows [0, Lq) from fp32 block sums.
@@ -165,7 +173,13 @@ void run_select_tokens(const hsa_params* p, int64_t Lq, int64_t Lk, const void* 
     }
     hsa::launch_topk_from_keys(rm, Lq, blocks, tkeys, p->B, p->m, p->k, indices, s);
   } else {
-    hsa::launch_select_tokens(rm, Lq, q_idx, k_idx, blocks, p->B, p->m, p->k, p->d_idx, indices, s);
+    // CUDA-core scoring: the row's candidates (at most m*B, at most Lk) in shared memory
+    if (std::min<int64_t>(int64_t(p->m) * p->B, Lk) > kMaxCandidatesSmem) {
+      *ok = false;
+      return;
+    }
+    hsa::launch_select_tokens(rm, Lq, q_idx, k_idx, blocks, p->B, p->m, p->k, p->d_idx, indices,
+                              std::min<int64_t>(int64_t(p->m) * p->B, Lk), s);
   }
 }
 
@@ -183,6 +197,12 @@ int hsa_device_status(int reset) {
   const int b = hsa::score_wait_flag(reset != 0);
   if (a < 0 || b < 0) return HSA_ERR_CUDA;
   return a || b ? HSA_ERR_TIMEOUT : HSA_OK;
+}
+
+int hsa_debug_inject_lost_arrival(int on) {
+  if (int e = check_device()) return e;
+  if (!hsa::attn_set_inject(on != 0) || !hsa::score_set_inject(on != 0)) return HSA_ERR_CUDA;
+  return HSA_OK;
 }
 
 const char* hsa_status_string(int status) {
@@ -278,14 +298,9 @@ int hsa_sparse_attn(const hsa_params* p, int64_t Lq, int64_t Lk, const hsa_bf16*
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(indices) || !aligned16(O))
     return HSA_ERR_ARG;
   if (int e = check_device()) return e;
-  if (hsa::tc_attn_supported(p->H, p->d, Lq, Lk)) {
-    if (!hsa::launch_sparse_attn_tc(Lq, Q, K, V, indices, Lk, p->k, p->H, softmax_scale(p), O, stream))
-      return HSA_ERR_CUDA;
-  } else {
-    hsa::RowMap rm{Lq, Lk, nullptr, 0};
-    hsa::launch_sparse_attn_simple(rm, Lq, Q, K, V, indices, p->k, p->H, p->d, softmax_scale(p), O,
-                                   stream);
-  }
+  if (!hsa::tc_attn_supported(p->H, p->d, Lq, Lk)) return HSA_ERR_ARG;
+  if (!hsa::launch_sparse_attn_tc(Lq, Q, K, V, indices, Lk, p->k, p->H, p->d, softmax_scale(p), O, stream))
+    return HSA_ERR_CUDA;
   return launch_status();
 }
 
@@ -342,7 +357,7 @@ int hsa_decode_step(const hsa_params* p, int32_t batch, int64_t capacity, int32_
                     cudaStream_t stream) {
   size_t need = 0;
   if (int e = hsa_decode_workspace_size(p, batch, capacity, &need)) return e;
-  if (capacity / p->B > kMaxCandidates || capacity > (int64_t(1) << 31) - 1) return HSA_ERR_ARG;
+  if (capacity / p->B > kMaxBlocks || capacity > (int64_t(1) << 31) - 1) return HSA_ERR_ARG;
   if (batch == 0) return HSA_OK;
   const void* ptrs[] = {k_idx_cache, K_cache, V_cache, ksum_cache, q_idx_new,
                         k_idx_new, Q_new, K_new, V_new, O};
@@ -363,32 +378,27 @@ int hsa_decode_step(const hsa_params* p, int32_t batch, int64_t capacity, int32_
   // The step's kernels are programmatic dependent launches: each may begin
   // launching while its predecessor runs, and waits for it before touching
   // memory (griddepcontrol), which hides the launch gaps of a short step.
-  // 1. append the new token (and the block sum of a block it completes)
-  hsa::launch_decode_append(batch, capacity, ctx_len, p->B, p->d_idx, p->d, k_idx_cache, K_cache,
-                            V_cache, ksum_cache, k_idx_new, K_new, V_new, stream);
-  // 2. block scores against the block-sum cache, top-m with the forced blocks
+  // 1. append the new token (and the block sum of a block it completes), in
+  //    the same kernel as 2. the block scores against the block-sum cache;
+  //    top-m with the forced blocks
   hsa::launch_decode_block_scores(batch, capacity, ctx_len, p->B, p->m, p->d_idx, q_idx_new, ksum_cache,
-                                  bkeys, nbc, stream);
+                                  bkeys, nbc, p->d, k_idx_cache, K_cache, V_cache, ksum_cache, k_idx_new,
+                                  K_new, V_new, stream);
   hsa::launch_topm_from_keys(rm, batch, bkeys, nbc, p->B, p->m, nbc > 2 ? nbc - 2 : 1, blocks, stream, true);
   // 3. token scores inside the kept blocks, top-k
   hsa::launch_decode_token_scores(batch, capacity, ctx_len, p->B, p->m, p->d_idx, blocks, q_idx_new,
                                   k_idx_cache, tkeys, stream);
   hsa::launch_topk_from_keys(rm, batch, blocks, tkeys, p->B, p->m, p->k, idx, stream, true);
-  // 4. attention over the kept tokens: parts of each query on the tensor cores, then combined
-  if (hsa::tc_attn_supported(p->H, p->d, batch, capacity)) {
-    float* opart = reinterpret_cast<float*>(ws + w.opart);
-    float* mpart = reinterpret_cast<float*>(ws + w.mpart);
-    float* lpart = reinterpret_cast<float*>(ws + w.lpart);
-    if (!hsa::launch_sparse_attn_tc_split(batch, Q_new, K_cache, V_cache, idx, capacity, p->k, p->H,
-                                          softmax_scale(p), w.parts, opart, mpart, lpart, stream, true))
-      return HSA_ERR_CUDA;
-    hsa::launch_decode_combine(batch, capacity, ctx_len, p->H, p->d, w.parts, opart, mpart, lpart, O, stream);
-  } else {
-    hsa::launch_sparse_attn_simple(rm, batch, Q_new, K_cache, V_cache, idx, p->k, p->H, p->d,
-                                   softmax_scale(p), O, stream, true);
-  }
-  // 5. the sequences grow by one token
-  hsa::launch_decode_advance(batch, capacity, ctx_len, stream);
+  // 4. attention over the kept tokens: parts of each query on the tensor cores,
+  //    then combined; 5. the combine also grows each sequence by one token
+  if (!hsa::tc_attn_supported(p->H, p->d, batch, capacity)) return HSA_ERR_ARG;
+  float* opart = reinterpret_cast<float*>(ws + w.opart);
+  float* mpart = reinterpret_cast<float*>(ws + w.mpart);
+  float* lpart = reinterpret_cast<float*>(ws + w.lpart);
+  if (!hsa::launch_sparse_attn_tc_split(batch, Q_new, K_cache, V_cache, idx, capacity, p->k, p->H, p->d,
+                                        softmax_scale(p), w.parts, opart, mpart, lpart, stream, true))
+    return HSA_ERR_CUDA;
+  hsa::launch_decode_combine(batch, capacity, ctx_len, p->H, p->d, w.parts, opart, mpart, lpart, O, stream);
   return launch_status();
 }
 

@@ -6,26 +6,33 @@
 // Orientation: the kept keys, not the heads, are the MMA's M dimension, so
 // every UMMA is a full 128-row tile whatever H is:
 //   S^T[key][h] = Ktile[key][:] . Q[h][:]        (A = gathered K rows, K-major;
-//                                                  B = the query's H x d block)
+//                                                  B = the query's heads, K-major)
 //   O^T[c][h]  += Vtile[key][c] . P^T[key][h]     (A = gathered V rows read
 //                                                  MN-major; B = P^T, MN-major)
+// A launch covers up to 64 heads (HP = 16, 32 or 64 MMA columns); more heads
+// take one launch per group of 64. Head dimension d = 128, or d = 64 with the
+// upper 64 rows of V^T read from a zero tile (O^T rows 64..127 stay 0).
+//
 // Per CTA (persistent over queries) the warp roles form a pipeline:
-//   warps 0..6   producers: Q tile per query by TMA; the K / V rows of each
-//                128-key tile by cp.async straight into the 128B-swizzled
-//                layout UMMA reads (row gathers through the LSU sustain far
-//                more bandwidth than TMA's four-row gathers);
-//   warp 7       MMA issuer (one thread): S^T of tile g, then O^T of tile g-1;
-//   warps 8..23  four softmax warpgroups, warpgroup w owning heads
-//                [w*H/4, (w+1)*H/4): thread = TMEM lane = key row of the tile.
+//   warps 0..3   producers: cp.async gathers of the kept K and V rows of each
+//                128-key tile straight into the 128B-swizzled layout UMMA
+//                reads (lane l loads the index of row 32w+l once per tile and
+//                the copying lanes take it by shuffle); warp 0 also copies
+//                each query's rows of Q (rows past its heads zero-filled);
+//   warp 4       S issuer: S^T of tile g;
+//   warp 5       PV issuer: O^T of tile g, so a barrier probe queued behind
+//                one kind of MMA never holds up the other;
+//   warps 6..21  four softmax warpgroups, warpgroup w owning heads
+//                [w*HP/4, (w+1)*HP/4): thread = TMEM lane = key row of the tile.
 // Softmax runs in the exp2 domain with a per-head running maximum that is
 // only raised (and O^T, l rescaled) when a tile exceeds it by more than 2^8,
 // so the cross-thread max reduction happens on a query's first tile and
 // rarely after; the per-tile check is one hardware barrier reduction. P is
 // rounded to bf16 for the second MMA; accumulation is fp32.
 //
-// A barrier probe in the MMA-issuing thread costs about as much as an MMA
-// when MMAs are queued, so with two stages that thread waits on one barrier
-// per MMA group: "K tile landed and S buffer read" before S, "P written and V
+// A barrier probe in an MMA-issuing thread costs about as much as an MMA when
+// MMAs are queued, so with two stages each issuer waits on one barrier per
+// MMA group: "K tile landed and S buffer read" before S, "P written and V
 // tile landed" before PV, each counting the arrivals of both producers.
 //
 // Every mbarrier wait is bounded. Within a softmax warpgroup all four warps
@@ -36,32 +43,38 @@
 
 namespace hsa {
 
-__device__ int g_attn_err;  // set when a bounded wait gives up
+__device__ int g_attn_err;     // set when a bounded wait gives up
+__device__ int g_attn_inject;  // test hook: short waits and one lost arrival
 
 namespace {
 
 using namespace tc;
 
-constexpr int D = 128;       // head dim handled by this kernel
 constexpr int TILE = 128;    // kept keys per MMA tile (the M dimension)
 constexpr int NWG = 4;       // softmax warpgroups
+constexpr int NPW = 4;       // producer warps: one kept-index row per lane
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr long long kInjectWaitCycles = 1ll << 21;  // about a millisecond
 
-template <int HP, int NPW>
+template <int HP, int DH>
 struct Cfg {
   static constexpr int NS = HP <= 32 ? 3 : 2;       // K/V pipeline stages
   static constexpr int HH = HP / NWG;               // heads per softmax warpgroup
   static constexpr int NSW = 4 * NWG;               // softmax warps
-  static constexpr int NWARPS = NPW + 1 + NSW;
-  static constexpr int KV_BYTES = TILE * D * 2;     // one K or V tile: 32 KB
-  static constexpr int Q_BYTES = HP * D * 2;        // one query's heads
+  static constexpr int NWARPS = NPW + 2 + NSW;      // + S issuer + PV issuer
+  static constexpr int KV_BYTES = TILE * DH * 2;    // one K or V tile
+  static constexpr int Q_BYTES = HP * DH * 2;       // one query's heads
   static constexpr int P_ROW = HP * 2;              // bytes of one P^T row (<= 128)
   static constexpr int P_BYTES = TILE * P_ROW;
+  static constexpr int Z_BYTES = DH == 64 ? TILE * 128 : 0;  // zero upper half of V^T
+  static constexpr int CPR = DH / 8;                // 16-byte chunks per K/V/Q row
+  static constexpr int RPI = 32 / CPR;              // rows per warp-wide copy
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + NS * KV_BYTES;
   static constexpr int OFF_Q = OFF_V + NS * KV_BYTES;
   static constexpr int OFF_P = OFF_Q + 2 * Q_BYTES;
-  static constexpr int SMEM = OFF_P + 2 * P_BYTES + 1024;  // + alignment slack
+  static constexpr int OFF_Z = OFF_P + 2 * P_BYTES;
+  static constexpr int SMEM = OFF_Z + Z_BYTES + 1024;  // + alignment slack
   static constexpr int TMEM_COLS = 4 * HP < 32 ? 32 : 4 * HP;
   static constexpr uint32_t P_SWZ = P_ROW == 128 ? kSw128 : P_ROW == 64 ? kSw64 : kSw32;
 };
@@ -78,18 +91,20 @@ struct Bars {
 
 // Work description of one launch. Query q's kept indices are idx[q][0..k);
 // its K/V rows start at row q * kv_stride (0: one K/V shared by all queries).
+// The launch covers heads [h0, h0 + nh) of the H heads of each Q / O row.
 // Each query is cut into items_per_query parts of tiles_per_item 128-key
 // tiles; with one part per query the kernel writes normalised O, otherwise
 // every part w = q * items_per_query + s writes its unnormalised O^T, running
 // maximum and row sum for a later combination.
 struct AttnArgs {
+  const uint16_t* Q;
   const int32_t* idx;
-  int Lq, Lk, k, H;
+  int Lq, Lk, k, H, h0, nh;
   float scale_log2;
   int64_t kv_stride;
   int items_per_query, tiles_per_item;
   uint16_t* O;
-  float *Opart, *mpart, *lpart;  // [items][H][D], [items][H], [items][H]
+  float *Opart, *mpart, *lpart;  // [items][H][d], [items][H], [items][H]
 };
 
 namespace {
@@ -98,7 +113,10 @@ namespace {
 // failure, so one lost arrival cannot keep any warp spinning for long.
 HSA_DEV bool wait_bar(uint64_t* bar, uint32_t parity, bool& dead) {
   if (dead) return false;
-  if (mbar_wait_bounded(bar, parity, &g_attn_err)) return true;
+  if (mbar_try_wait(bar, parity)) return true;
+  // the limit is read only on this slow path: the test hook shortens it
+  const long long lim = *(volatile int*)&g_attn_inject ? kInjectWaitCycles : kWaitCycles;
+  if (mbar_wait_bounded(bar, parity, &g_attn_err, lim)) return true;
   dead = true;
   return false;
 }
@@ -128,6 +146,24 @@ HSA_DEV bool wg_or(int id, bool v) {
       : "r"(id), "r"(uint32_t(v))
       : "memory");
   return out != 0;
+}
+
+// x0,x1 = fma(x0,x1 ; s,s ; c0,c1) as one packed f32x2 instruction (round to nearest)
+HSA_DEV void ffma2(float& x0, float& x1, float s, float c0, float c1) {
+  asm("{\n .reg .b64 ra, rb, rc;\n mov.b64 ra, {%0, %1};\n mov.b64 rb, {%2, %2};\n"
+      " mov.b64 rc, {%3, %4};\n fma.rn.f32x2 ra, ra, rb, rc;\n mov.b64 {%0, %1}, ra;\n}"
+      : "+f"(x0), "+f"(x1) : "f"(s), "f"(c0), "f"(c1));
+}
+// a0,a1 += b0,b1 as one packed f32x2 instruction (round to nearest)
+HSA_DEV void fadd2(float& a0, float& a1, float b0, float b1) {
+  asm("{\n .reg .b64 ra, rb;\n mov.b64 ra, {%0, %1};\n mov.b64 rb, {%2, %3};\n"
+      " add.rn.f32x2 ra, ra, rb;\n mov.b64 {%0, %1}, ra;\n}"
+      : "+f"(a0), "+f"(a1) : "f"(b0), "f"(b1));
+}
+HSA_DEV float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 HSA_DEV float redux_max(float v) {
@@ -169,6 +205,38 @@ HSA_DEV int transpose_head(int lane, int i) {
   return lane >> shift;
 }
 
+// Tiles of a query (or part) given where its kept list ends: the last valid
+// index position is found from the last 128 entries, fetched one query ahead
+// by the caller, or by a backwards search in the rare row whose tail is all
+// padding. Warp-collective; every lane returns the same count.
+struct TailScan {
+  bool vec;
+  int s0;
+  HSA_DEV int4 window(const int32_t* idx, int q, int k) const {
+    return vec ? __ldg(reinterpret_cast<const int4*>(idx + int64_t(q) * k + s0) + (threadIdx.x & 31))
+               : make_int4(-1, -1, -1, -1);
+  }
+  HSA_DEV int last_valid(int4 win, const int32_t* row, int k, int Lk) const {
+    const int lane = threadIdx.x & 31;
+    int last = -1;
+    if (vec) {
+      if (win.x >= 0 && win.x < Lk) last = s0 + 4 * lane;
+      if (win.y >= 0 && win.y < Lk) last = s0 + 4 * lane + 1;
+      if (win.z >= 0 && win.z < Lk) last = s0 + 4 * lane + 2;
+      if (win.w >= 0 && win.w < Lk) last = s0 + 4 * lane + 3;
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) last = max(last, __shfl_xor_sync(kFull, last, o));
+    for (int c0 = (vec ? s0 : k) - 32; last < 0 && c0 > -32; c0 -= 32) {  // backwards, 32 at a time
+      const int pp = c0 + lane;
+      const int j = pp >= 0 ? __ldg(row + pp) : -1;
+      const unsigned v = __ballot_sync(kFull, j >= 0 && j < Lk);
+      if (v) last = c0 + 31 - __clz(v);
+    }
+    return last;
+  }
+};
+
 // N consecutive 32-bit TMEM columns of this warp's 32 lanes (N = 4, 8, 16).
 template <int N>
 HSA_DEV void tmem_ld_cols(uint32_t taddr, float (&v)[N]) {
@@ -191,11 +259,10 @@ HSA_DEV void tmem_st_cols(uint32_t taddr, const float (&v)[N]) {
   tmem_wait_st();
 }
 
-template <int HP, int NPW>
-__global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_kernel(
-    const __grid_constant__ CUtensorMap qmap, const uint16_t* __restrict__ K, const uint16_t* __restrict__ V,
-    const AttnArgs a) {
-  using C = Cfg<HP, NPW>;
+template <int HP, int DH>
+__global__ void __launch_bounds__(32 * Cfg<HP, DH>::NWARPS, 1) sparse_attn_tc_kernel(
+    const uint16_t* __restrict__ K, const uint16_t* __restrict__ V, const AttnArgs a) {
+  using C = Cfg<HP, DH>;
   const int32_t* __restrict__ idx = a.idx;
   const int Lk = a.Lk, k = a.k, H = a.H;
   const float scale_log2 = a.scale_log2;
@@ -212,13 +279,14 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
   __shared__ float lsum[HP];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nh = a.nh;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NS; ++s) {
       mbar_init(&bars.kfull[s], NPW * 32); mbar_init(&bars.kempty[s], 1);
       mbar_init(&bars.vfull[s], NPW * 32); mbar_init(&bars.vempty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&bars.qfull[b], 1); mbar_init(&bars.qempty[b], 1 + C::NSW);
+      mbar_init(&bars.qfull[b], 32 + 1); mbar_init(&bars.qempty[b], 2 + C::NSW);
       mbar_init(&bars.sfull[b], 1); mbar_init(&bars.sempty[b], C::NSW);
       mbar_init(&bars.pfull[b], C::NSW); mbar_init(&bars.pempty[b], 1);
       mbar_init(&bars.sgo[b], NPW * 32 + C::NSW); mbar_init(&bars.pgo[b], NPW * 32 + C::NSW);
@@ -226,8 +294,13 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
       for (int u = 0; u < C::NSW; ++u) mbar_arrive(&bars.sgo[b]);
       mbar_init(&bars.ofull[b], 1); mbar_init(&bars.oempty[b], C::NSW);
     }
-    mbar_init(&bars.done, 1);
+    mbar_init(&bars.done, 2);
     fence_barrier_init();
+  }
+  if constexpr (C::Z_BYTES > 0) {
+    for (int e = threadIdx.x; e < C::Z_BYTES / 16; e += 32 * C::NWARPS)
+      reinterpret_cast<uint4*>(sm + C::OFF_Z)[e] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();  // written here, read by the MMA
   }
   if (warp == NPW) { tmem_alloc(&tmem_base, C::TMEM_COLS); tmem_relinquish(); }
   tc_fence_before();
@@ -242,131 +315,87 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
 
   if (warp < NPW) {
     // ------------------------------------------------------------ producers
-    // Producer thread p copies the (row, 16-byte chunk) pairs p, p + 32*NPW, ...
-    // of each K and V tile with cp.async into the 128B-swizzled layout.
-    constexpr int PT = NPW * 32, PER = (TILE * 16 + PT - 1) / PT;
-    const int p = threadIdx.x;
-    if (p == 0) prefetch_tmap(&qmap);
-    // The tile count of a query needs its last valid index position: the
-    // row is searched backwards 128 entries at a time, and the last 128
-    // entries of the next query's row are fetched one query ahead, so the
-    // usual case (a valid tail) costs no exposed load latency.
-    const bool vec = (k & 3) == 0 && k >= 128;
-    const int s0 = vec ? k - 128 : 0;  // start of the last 128-entry window
-    auto tail_window = [&](int q) -> int4 {
-      return vec ? __ldg(reinterpret_cast<const int4*>(idx + int64_t(q) * k + s0) + lane) : make_int4(-1, -1, -1, -1);
-    };
-    int4 pre = blockIdx.x < n_items ? tail_window(blockIdx.x / ipq) : make_int4(-1, -1, -1, -1);
+    static_assert(TILE == 32 * NPW, "one kept-index row per producer lane");
+    // the copy of (row 32 * warp + RPI * u + rsub, chunk cpk) takes the row's
+    // index from lane RPI * u + rsub
+    const int rsub = lane / C::CPR, cpk = lane % C::CPR;
+    // shared-memory offset of (row 32 * warp + rsub, chunk cpk) in the
+    // 128B-swizzled K-major tile, before the swizzle of the chunk
+    const uint32_t dbase = (cpk >> 3) * (TILE * 128) + (32 * warp + rsub) * 128;
+    const TailScan ts{(k & 3) == 0 && k >= 128, ((k & 3) == 0 && k >= 128) ? k - 128 : 0};
+    int4 pre = blockIdx.x < n_items ? ts.window(idx, blockIdx.x / ipq, k) : make_int4(-1, -1, -1, -1);
+    const bool inject = *(volatile int*)&g_attn_inject != 0;
     uint32_t g = 0, qn = 0;
     for (int w = blockIdx.x; w < n_items && !dead; w += gridDim.x, ++qn) {
       const int q = w / ipq, part = w - q * ipq;
       const int32_t* row = idx + int64_t(q) * k;
-      const uint4* Kq = reinterpret_cast<const uint4*>(K + int64_t(q) * a.kv_stride * D);
-      const uint4* Vq = reinterpret_cast<const uint4*>(V + int64_t(q) * a.kv_stride * D);
+      const uint4* Kq = reinterpret_cast<const uint4*>(K + int64_t(q) * a.kv_stride * DH);
+      const uint4* Vq = reinterpret_cast<const uint4*>(V + int64_t(q) * a.kv_stride * DH);
       const int4 win = pre;
-      if (w + int(gridDim.x) < n_items) pre = tail_window((w + gridDim.x) / ipq);
-      int last = -1;  // tiles = ceil((last valid position + 1) / TILE)
-      if (vec) {
-        if (win.x >= 0 && win.x < Lk) last = s0 + 4 * lane;
-        if (win.y >= 0 && win.y < Lk) last = s0 + 4 * lane + 1;
-        if (win.z >= 0 && win.z < Lk) last = s0 + 4 * lane + 2;
-        if (win.w >= 0 && win.w < Lk) last = s0 + 4 * lane + 3;
-      }
-#pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) last = max(last, __shfl_xor_sync(kFull, last, o));
-      for (int c0 = (vec ? s0 : k) - 32; last < 0 && c0 > -32; c0 -= 32) {  // backwards, 32 at a time
-        const int pp = c0 + lane;
-        const int j = pp >= 0 ? __ldg(row + pp) : -1;
-        const unsigned v = __ballot_sync(kFull, j >= 0 && j < Lk);
-        if (v) last = c0 + 31 - __clz(v);
-      }
+      if (w + int(gridDim.x) < n_items) pre = ts.window(idx, (w + gridDim.x) / ipq, k);
+      const int last = ts.last_valid(win, row, k, Lk);
       const int t0 = part * tpi;                                  // this item's tiles
       const int nt = max(0, min((last + TILE) / TILE, t0 + tpi) - t0);
       const int qb = qn & 1;
+      // warp 0: this query's HP head rows of Q (rows past its nh heads: zeros)
+      // and its tile count; the other producers go straight on to its tiles
       if (warp == 0) {
         if (!wait_warp(&bars.qempty[qb], ((qn >> 1) & 1) ^ 1, dead)) break;
         if (lane == 0) {
           qinfo[qb][0] = t0;
           qinfo[qb][1] = nt;
-          mbar_arrive_expect_tx(&bars.qfull[qb], C::Q_BYTES);
-          uint8_t* qt = sm + C::OFF_Q + qb * C::Q_BYTES;
-          tma_load_2d(qt, &qmap, &bars.qfull[qb], 0, q * H);
-          tma_load_2d(qt + HP * 128, &qmap, &bars.qfull[qb], 64, q * H);
+          mbar_arrive(&bars.qfull[qb]);  // releases qinfo
         }
+        const uint32_t qt = smem_u32(sm + C::OFF_Q + qb * C::Q_BYTES);
+        const uint4* qsrc = reinterpret_cast<const uint4*>(a.Q) + (int64_t(q) * H + a.h0) * C::CPR;
+        for (int e = lane; e < HP * C::CPR; e += 32) {
+          const int h = e / C::CPR, c = e % C::CPR;
+          const bool live = h < nh;
+          cp_async16_zfill(qt + (c >> 3) * (HP * 128) + swz_offset(h, c & 7, 128),
+                           live ? qsrc + h * C::CPR + c : qsrc, live);
+        }
+        cp_async_arrive(&bars.qfull[qb]);
       }
       for (int i = 0; i < nt && !dead; ++i, ++g) {
         const int s = g % C::NS;
         const uint32_t ph = (g / C::NS) & 1;
-        int jr[PER];
-        uint32_t dst[PER];
-#pragma unroll
-        for (int u = 0; u < PER; ++u) {
-          const int e = p + u * PT, r = (e >> 4) & (TILE - 1), c = e & 15;
-          const int pos = (t0 + i) * TILE + r;
-          const int j = (e < TILE * 16 && pos < k) ? __ldg(row + pos) : -1;
-          jr[u] = ((j >= 0 && j < Lk) ? j : 0) * (D / 8) + c;   // 16-byte units
-          dst[u] = (c >> 3) * (TILE * 128) + swz_offset(r, c & 7, 128);
-        }
+        // lane l fetches the kept index of row 32 * warp + l
+        const int pos = (t0 + i) * TILE + 32 * warp + lane;
+        const int jv = pos < k ? __ldg(row + pos) : -1;
+        const int jc = ((jv >= 0 && jv < Lk) ? jv : 0) * C::CPR;  // row start, 16-byte units
         // with two stages, a K stage is free once S of the tile two back is
         // done (sfull), a V stage once its PV is done (pempty)
         if (!wait_warp(C::NS == 2 ? &bars.sfull[s] : &bars.kempty[s], ph ^ 1, dead)) break;
-        const uint32_t kt = smem_u32(sm + C::OFF_K + s * C::KV_BYTES);
+        const uint32_t kt = smem_u32(sm + C::OFF_K + s * C::KV_BYTES) + dbase;
+        int jr[32 / C::RPI];
 #pragma unroll
-        for (int u = 0; u < PER; ++u)
-          if (p + u * PT < TILE * 16) cp_async16(kt + dst[u], Kq + jr[u]);
-        cp_async_arrive(C::NS == 2 ? &bars.sgo[s] : &bars.kfull[s]);
+        for (int u = 0; u < 32 / C::RPI; ++u) {
+          const int rr = C::RPI * u + rsub;
+          jr[u] = __shfl_sync(kFull, jc, rr) + cpk;
+          cp_async16(kt + u * (C::RPI * 128) + ((uint32_t((cpk & 7) ^ (rr & 7))) << 4), Kq + jr[u]);
+        }
+        // test hook: one producer's K arrival on the first tile of CTA 0 is lost
+        if (!(inject && blockIdx.x == 0 && g == 0 && warp == 0 && lane == 0))
+          cp_async_arrive(C::NS == 2 ? &bars.sgo[s] : &bars.kfull[s]);
         if (!wait_warp(C::NS == 2 ? &bars.pempty[s] : &bars.vempty[s], ph ^ 1, dead)) break;
-        const uint32_t vt = smem_u32(sm + C::OFF_V + s * C::KV_BYTES);
+        const uint32_t vt = smem_u32(sm + C::OFF_V + s * C::KV_BYTES) + dbase;
 #pragma unroll
-        for (int u = 0; u < PER; ++u)
-          if (p + u * PT < TILE * 16) cp_async16(vt + dst[u], Vq + jr[u]);
+        for (int u = 0; u < 32 / C::RPI; ++u)
+          cp_async16(vt + u * (C::RPI * 128) + ((uint32_t((cpk & 7) ^ ((C::RPI * u + rsub) & 7))) << 4), Vq + jr[u]);
         cp_async_arrive(C::NS == 2 ? &bars.pgo[s] : &bars.vfull[s]);
       }
     }
     cp_async_wait_all();  // every copy has landed before the CTA may exit
-    if (warp == 0 && lane == 0) {
-      bool d2 = false;
-      for (uint32_t t = (qn >= 2 ? qn - 2 : 0); t < qn; ++t) wait_bar(&bars.qfull[t & 1], (t >> 1) & 1, d2);
-    }
   } else if (warp == NPW) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ S issuer
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_bf16(128, HP, false, false);
-      constexpr uint32_t id_o = idesc_bf16(128, HP, true, true);
-      uint32_t g = 0, qn = 0, oq = 0;
-      struct Pend { uint32_t g, ob, oq; bool first, last, valid; } prev{0, 0, 0, false, false, false};
-      auto issue_pv = [&](const Pend& t) {
-        const int pb = t.g & 1, s = t.g % C::NS;
-        if constexpr (C::NS == 2) {
-          // one wait per tile: P written and V landed
-          if (!wait_bar(&bars.pgo[pb], (t.g >> 1) & 1, dead)) return;
-        } else {
-          if (!wait_bar(&bars.pfull[pb], (t.g >> 1) & 1, dead)) return;
-          if (!wait_bar(&bars.vfull[s], (t.g / C::NS) & 1, dead)) return;
-        }
-        if (t.first && !wait_bar(&bars.oempty[t.ob], ((t.oq >> 1) & 1) ^ 1, dead)) return;
-        // the V rows landed by cp.async (generic proxy) are read by the MMA
-        // (async proxy): order them across proxies after the acquire above
-        fence_proxy_async_smem();
-        tc_fence_after();
-        const uint64_t a0 = smem_desc(smem_u32(sm + C::OFF_V + s * C::KV_BYTES), TILE * 128, 1024, kSw128);
-        const uint64_t b0 = smem_desc(smem_u32(sm + C::OFF_P + pb * C::P_BYTES), 16384, 8 * C::P_ROW, C::P_SWZ);
-        const uint32_t d = tmem + 2 * HP + t.ob * HP;
-        const uint32_t alo = uint32_t(a0), ahi = uint32_t(a0 >> 32), blo = uint32_t(b0), bhi = uint32_t(b0 >> 32);
-#pragma unroll
-        for (int ks = 0; ks < TILE / 16; ++ks)
-          mma_bf16_split(d, alo + ((ks * 2048) >> 4), ahi, blo + ((ks * 16 * C::P_ROW) >> 4), bhi, id_o,
-                         (t.first && ks == 0) ? 0u : 1u);
-        if (C::NS != 2) mma_commit(&bars.vempty[s]);
-        mma_commit(&bars.pempty[pb]);
-        if (t.last) mma_commit(&bars.ofull[t.ob]);
-      };
+      uint32_t g = 0, qn = 0;
       for (int w = blockIdx.x; w < n_items && !dead; w += gridDim.x, ++qn) {
         const int qb = qn & 1;
         if (!wait_bar(&bars.qfull[qb], (qn >> 1) & 1, dead)) break;
         const int nt = qinfo[qb][1];
         if (nt == 0) { mbar_arrive(&bars.qempty[qb]); continue; }
-        const uint32_t ob = oq & 1;
         const uint64_t qd0 = smem_desc(smem_u32(sm + C::OFF_Q + qb * C::Q_BYTES), 16, 1024, kSw128);
         const uint32_t qlo = uint32_t(qd0), qhi = uint32_t(qd0 >> 32);
         for (int i = 0; i < nt && !dead; ++i, ++g) {
@@ -383,26 +412,70 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
           const uint64_t kd0 = smem_desc(smem_u32(sm + C::OFF_K + s * C::KV_BYTES), 16, 1024, kSw128);
           const uint32_t klo = uint32_t(kd0), khi = uint32_t(kd0 >> 32);
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks)
+          for (int ks = 0; ks < DH / 16; ++ks)
             mma_bf16_split(tmem + sb * HP, klo + (((ks / 4) * TILE * 128 + (ks % 4) * 32) >> 4), khi,
                            qlo + (((ks / 4) * HP * 128 + (ks % 4) * 32) >> 4), qhi, id_s, ks > 0 ? 1u : 0u);
           if (C::NS != 2) mma_commit(&bars.kempty[s]);
           mma_commit(&bars.sfull[sb]);
           if (i == nt - 1) mma_commit(&bars.qempty[qb]);
-          if (prev.valid) issue_pv(prev);
-          prev = Pend{g, ob, oq, i == 0, i == nt - 1, true};
+        }
+      }
+      mma_commit(&bars.done);  // counts once, when this thread's MMAs are complete
+      bool d2 = false;
+      wait_bar(&bars.done, 0, d2);
+    }
+    __syncwarp();
+  } else if (warp == NPW + 1) {
+    // ------------------------------------------------------------ PV issuer
+    if (lane == 0) {
+      constexpr uint32_t id_o = idesc_bf16(128, HP, true, true);
+      uint32_t g = 0, qn = 0, oq = 0;
+      for (int w = blockIdx.x; w < n_items && !dead; w += gridDim.x, ++qn) {
+        const int qb = qn & 1;
+        if (!wait_bar(&bars.qfull[qb], (qn >> 1) & 1, dead)) break;
+        const int nt = qinfo[qb][1];
+        mbar_arrive(&bars.qempty[qb]);  // the tile count is all this thread reads of the query
+        if (nt == 0) continue;
+        const uint32_t ob = oq & 1;
+        for (int i = 0; i < nt && !dead; ++i, ++g) {
+          const int pb = g & 1, s = g % C::NS;
+          if constexpr (C::NS == 2) {
+            // one wait per tile: P written and V landed
+            if (!wait_bar(&bars.pgo[pb], (g >> 1) & 1, dead)) break;
+          } else {
+            if (!wait_bar(&bars.pfull[pb], (g >> 1) & 1, dead)) break;
+            if (!wait_bar(&bars.vfull[s], (g / C::NS) & 1, dead)) break;
+          }
+          if (i == 0 && !wait_bar(&bars.oempty[ob], ((oq >> 1) & 1) ^ 1, dead)) break;
+          // the V rows landed by cp.async (generic proxy) are read by the MMA
+          // (async proxy): order them across proxies after the acquire above
+          fence_proxy_async_smem();
+          tc_fence_after();
+          const uint32_t vs = smem_u32(sm + C::OFF_V + s * C::KV_BYTES);
+          // the second 64 rows of V^T: the tile's upper half, or the zero tile when d = 64
+          const uint32_t lbo = DH == 128 ? TILE * 128 : smem_u32(sm + C::OFF_Z) - vs;
+          const uint64_t a0 = smem_desc(vs, lbo, 1024, kSw128);
+          const uint64_t b0 = smem_desc(smem_u32(sm + C::OFF_P + pb * C::P_BYTES), 16384, 8 * C::P_ROW, C::P_SWZ);
+          const uint32_t d = tmem + 2 * HP + ob * HP;
+          const uint32_t alo = uint32_t(a0), ahi = uint32_t(a0 >> 32), blo = uint32_t(b0), bhi = uint32_t(b0 >> 32);
+#pragma unroll
+          for (int ks = 0; ks < TILE / 16; ++ks)
+            mma_bf16_split(d, alo + ((ks * 2048) >> 4), ahi, blo + ((ks * 16 * C::P_ROW) >> 4), bhi, id_o,
+                           (i == 0 && ks == 0) ? 0u : 1u);
+          if (C::NS != 2) mma_commit(&bars.vempty[s]);
+          mma_commit(&bars.pempty[pb]);
+          if (i == nt - 1) mma_commit(&bars.ofull[ob]);
         }
         ++oq;
       }
-      if (prev.valid && !dead) issue_pv(prev);
-      mma_commit(&bars.done);  // all issued MMAs complete before TMEM is released
+      mma_commit(&bars.done);
       bool d2 = false;
       wait_bar(&bars.done, 0, d2);
     }
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax / epilogue
-    const int sw = warp - NPW - 1, wg = sw >> 2;
+    const int sw = warp - NPW - 2, wg = sw >> 2;
     const int bar_id = 1 + wg;
     const int quad = warp & 3;              // TMEM lane quadrant this warp may access
     const int wq = quad;                    // slot of this warp in the warpgroup's scratch rows
@@ -418,15 +491,16 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
       const int t0 = qinfo[qb][0], nt = qinfo[qb][1];
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.qempty[qb]);
-      uint16_t* orow = a.O ? a.O + int64_t(q) * H * D : nullptr;
+      // this query's rows of O (head a.h0 + h0 + h of the launch's heads)
+      uint16_t* orow = a.O ? a.O + (int64_t(q) * H + a.h0) * DH : nullptr;
       if (nt == 0) {
         if (orow) {
 #pragma unroll
           for (int h = 0; h < HH; ++h)
-            if (h0 + h < H) orow[(h0 + h) * D + r] = 0;
-        } else if (r < HH && h0 + r < H) {  // an empty part: no weight in the combination
-          a.mpart[int64_t(w) * H + h0 + r] = -INFINITY;
-          a.lpart[int64_t(w) * H + h0 + r] = 0.f;
+            if (h0 + h < nh && r < DH) orow[(h0 + h) * DH + r] = 0;
+        } else if (r < HH && h0 + r < nh) {  // an empty part: no weight in the combination
+          a.mpart[int64_t(w) * H + a.h0 + h0 + r] = -INFINITY;
+          a.lpart[int64_t(w) * H + a.h0 + h0 + r] = 0.f;
         }
         continue;
       }
@@ -435,9 +509,9 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
       // m: running maximum per head (log2 units), or 0 while the head has
       // seen no valid key (its scores so far are all -inf, so 2^(x - 0) = 0);
       // `complete`: every real head of this warpgroup has a finite maximum.
-      float lp[HH], m[HH];
+      float lp[HH], nm[HH];  // nm: the running maximum, negated
 #pragma unroll
-      for (int h = 0; h < HH; ++h) { lp[h] = 0.f; m[h] = 0.f; }
+      for (int h = 0; h < HH; ++h) { lp[h] = 0.f; nm[h] = 0.f; }
       bool complete = false;
       bool quit = false;
       for (int i = 0; i < nt; ++i, ++g) {
@@ -460,15 +534,15 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
         const bool live = oks && valid;
         float tmax = -INFINITY;
 #pragma unroll
-        for (int h = 0; h < HH; ++h) {
-          x[h] = fmaf(x[h], scale_log2, -m[h]);
-          tmax = fmaxf(tmax, x[h]);
+        for (int h = 0; h < HH; h += 2) {
+          ffma2(x[h], x[h + 1], scale_log2, nm[h], nm[h + 1]);
+          tmax = fmax3(tmax, x[h], x[h + 1]);
         }
-        if (!live || h0 + HH > H) {
+        if (!live || h0 + HH > nh) {
           tmax = -INFINITY;
 #pragma unroll
           for (int h = 0; h < HH; ++h) {
-            if (!live || h0 + h >= H) x[h] = -INFINITY;
+            if (!live || h0 + h >= nh) x[h] = -INFINITY;
             tmax = fmaxf(tmax, x[h]);
           }
         }
@@ -479,7 +553,7 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
           // raise the running maxima of this warpgroup's heads to cover the tile
 #pragma unroll
           for (int h = 0; h < HH; ++h) {
-            const float wm = redux_max(x[h] + m[h]);  // the tile's scaled scores
+            const float wm = redux_max(x[h] - nm[h]);  // the tile's scaled scores
             if (lane == (h & 31)) red[wq][h0 + h] = wm;
           }
           wg_sync(bar_id);
@@ -496,9 +570,9 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
           for (int h = 0; h < HH; ++h) {
             const float n = mh[h0 + h];
             const float mn = n == -INFINITY ? 0.f : n;
-            x[h] += m[h] - mn;  // re-centre the exponents on the new maximum
-            m[h] = mn;
-            all = all && (n != -INFINITY || h0 + h >= H);
+            x[h] -= nm[h] + mn;  // re-centre the exponents on the new maximum
+            nm[h] = -mn;
+            all = all && (n != -INFINITY || h0 + h >= nh);
           }
           complete = all;
           if (i > 0) {
@@ -533,8 +607,7 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
 #pragma unroll
         for (int e = 0; e < HH / 2; ++e) {
           const float p0 = ex2(x[2 * e]), p1 = ex2(x[2 * e + 1]);
-          lp[2 * e] += p0;
-          lp[2 * e + 1] += p1;
+          fadd2(lp[2 * e], lp[2 * e + 1], p0, p1);
           w[e] = cvt_bf16x2(p0, p1);
         }
         if (okw) {
@@ -572,20 +645,20 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
         if (orow) {
 #pragma unroll
           for (int h = 0; h < HH; ++h) {
-            if (h0 + h < H) {
+            if (h0 + h < nh && r < DH) {
               const float l = lsum[h0 + h];
-              orow[(h0 + h) * D + r] = uint16_t(f32_to_bf16_rn(l > 0.f ? ov[h] / l : 0.f));
+              orow[(h0 + h) * DH + r] = uint16_t(f32_to_bf16_rn(l > 0.f ? ov[h] / l : 0.f));
             }
           }
         } else {
           // one part of a split query: unnormalised O^T, running maximum, row sum
-          float* op = a.Opart + int64_t(w) * H * D;
+          float* op = a.Opart + (int64_t(w) * H + a.h0) * DH;
 #pragma unroll
           for (int h = 0; h < HH; ++h)
-            if (h0 + h < H) op[(h0 + h) * D + r] = ov[h];
-          if (r < HH && h0 + r < H) {
-            a.mpart[int64_t(w) * H + h0 + r] = mh[h0 + r];
-            a.lpart[int64_t(w) * H + h0 + r] = lsum[h0 + r];
+            if (h0 + h < nh && r < DH) op[(h0 + h) * DH + r] = ov[h];
+          if (r < HH && h0 + r < nh) {
+            a.mpart[int64_t(w) * H + a.h0 + h0 + r] = mh[h0 + r];
+            a.lpart[int64_t(w) * H + a.h0 + h0 + r] = lsum[h0 + r];
           }
         }
       }
@@ -605,59 +678,66 @@ __global__ void __launch_bounds__(32 * Cfg<HP, NPW>::NWARPS, 1) sparse_attn_tc_k
   }
 }
 
-// 7 producer warps + 1 MMA warp + 16 softmax warps = 24 warps (6 per SM
-// sub-partition, 80 registers per thread).
-constexpr int kProducerWarps = 7;
-
-template <int HP>
-bool launch_hp(const void* Q, const void* K, const void* V, const AttnArgs& a, cudaStream_t s, bool pdl) {
-  CUtensorMap qm;
-  if (!make_tmap_2d(&qm, Q, uint64_t(a.Lq) * a.H, D, HP)) return false;
-  using C = Cfg<HP, kProducerWarps>;
-  auto kern = sparse_attn_tc_kernel<HP, kProducerWarps>;
+// 4 producer warps + 2 MMA-issuing warps + 16 softmax warps = 22 warps (80
+// registers per thread).
+template <int HP, int DH>
+bool launch_hp(const AttnArgs& a, const void* K, const void* V, cudaStream_t s, bool pdl) {
+  using C = Cfg<HP, DH>;
+  auto kern = sparse_attn_tc_kernel<HP, DH>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
     return false;
   const int64_t items = int64_t(a.Lq) * a.items_per_query;
   const int grid = int(items < num_sms() ? items : num_sms());
-  launch_kernel(pdl, kern, grid, 32 * C::NWARPS, C::SMEM, s, qm, static_cast<const uint16_t*>(K),
+  launch_kernel(pdl, kern, grid, 32 * C::NWARPS, C::SMEM, s, static_cast<const uint16_t*>(K),
                 static_cast<const uint16_t*>(V), a);
   return true;
 }
 
-bool launch_args(const void* Q, const void* K, const void* V, const AttnArgs& a, cudaStream_t s, bool pdl) {
-  count_launches(1);
-  if (a.H <= 16) return launch_hp<16>(Q, K, V, a, s, pdl);
-  if (a.H <= 32) return launch_hp<32>(Q, K, V, a, s, pdl);
-  return launch_hp<64>(Q, K, V, a, s, pdl);
+template <int DH>
+bool launch_group(const AttnArgs& a, const void* K, const void* V, cudaStream_t s, bool pdl) {
+  if (a.nh <= 16) return launch_hp<16, DH>(a, K, V, s, pdl);
+  if (a.nh <= 32) return launch_hp<32, DH>(a, K, V, s, pdl);
+  return launch_hp<64, DH>(a, K, V, s, pdl);
+}
+
+// One launch per group of up to 64 heads.
+bool launch_args(AttnArgs a, int d, const void* K, const void* V, cudaStream_t s, bool pdl) {
+  for (int h0 = 0; h0 < a.H; h0 += 64) {
+    a.h0 = h0;
+    a.nh = a.H - h0 < 64 ? a.H - h0 : 64;
+    count_launches(1);
+    const bool ok = d == 128 ? launch_group<128>(a, K, V, s, pdl) : launch_group<64>(a, K, V, s, pdl);
+    if (!ok) return false;
+  }
+  return true;
 }
 
 }  // namespace
 
 bool tc_attn_supported(int H, int d, int64_t Lq, int64_t Lk) {
-  const int hp = H <= 16 ? 16 : H <= 32 ? 32 : 64;
-  // the Q box (hp rows) must fit inside the [Lq*H][d] tensor map
-  return d == 128 && H >= 1 && H <= 64 && Lq * H >= hp && Lq * H < (int64_t(1) << 31) &&
-         Lk < (int64_t(1) << 31);
+  return (d == 128 || d == 64) && H >= 1 && Lq * H < (int64_t(1) << 31) && Lk < (int64_t(1) << 31);
 }
 
 bool launch_sparse_attn_tc(int64_t Lq, const void* Q, const void* K, const void* V, const int32_t* idx,
-                           int64_t Lk, int k, int H, float scale, void* O, cudaStream_t s) {
+                           int64_t Lk, int k, int H, int d, float scale, void* O, cudaStream_t s) {
   if (Lq == 0) return true;
   AttnArgs a{};
+  a.Q = static_cast<const uint16_t*>(Q);
   a.idx = idx; a.Lq = int(Lq); a.Lk = int(Lk); a.k = k; a.H = H;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.kv_stride = 0;
   a.items_per_query = 1;
   a.tiles_per_item = (k + TILE - 1) / TILE;
   a.O = static_cast<uint16_t*>(O);
-  return launch_args(Q, K, V, a, s, false);
+  return launch_args(a, d, K, V, s, false);
 }
 
 bool launch_sparse_attn_tc_split(int batch, const void* Q, const void* Kc, const void* Vc, const int32_t* idx,
-                                 int64_t capacity, int k, int H, float scale, int parts, float* Opart,
+                                 int64_t capacity, int k, int H, int d, float scale, int parts, float* Opart,
                                  float* mpart, float* lpart, cudaStream_t s, bool pdl) {
   if (batch == 0) return true;
   AttnArgs a{};
+  a.Q = static_cast<const uint16_t*>(Q);
   a.idx = idx; a.Lq = batch; a.Lk = int(capacity); a.k = k; a.H = H;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.kv_stride = capacity;
@@ -665,7 +745,7 @@ bool launch_sparse_attn_tc_split(int batch, const void* Q, const void* Kc, const
   a.tiles_per_item = ((k + TILE - 1) / TILE + parts - 1) / parts;
   a.O = nullptr;
   a.Opart = Opart; a.mpart = mpart; a.lpart = lpart;
-  return launch_args(Q, Kc, Vc, a, s, pdl);
+  return launch_args(a, d, Kc, Vc, s, pdl);
 }
 
 // Host side: whether a bounded wait of this kernel gave up on the current
@@ -678,6 +758,12 @@ int attn_wait_flag(bool reset) {
     if (cudaMemcpyToSymbol(g_attn_err, &zero, sizeof zero) != cudaSuccess) return -1;
   }
   return v != 0;
+}
+
+// Host side: turn the attention's test hook on or off on the current device.
+bool attn_set_inject(bool on) {
+  const int v = on ? 1 : 0;
+  return cudaMemcpyToSymbol(g_attn_inject, &v, sizeof v) == cudaSuccess;
 }
 
 }  // namespace hsa

@@ -1,39 +1,42 @@
-// Decode-step helpers: append one token per sequence to the caller's caches
-// (writing the block sum of a block the token completes) and advance the
-// per-sequence lengths once the step's selection and attention are queued.
+// Decode-step kernels: block scores of each sequence's new query (whose first
+// CTA also appends the new token to the caller's caches and writes the block
+// sum of a block the token completes), token scores inside the kept blocks,
+// and the combination of a split attention's parts (which also advances the
+// per-sequence lengths once every earlier kernel of the step has read them).
+#include <algorithm>
+
 #include "kernels.cuh"
 
 namespace hsa {
 
-template <int DI, int DA>
-__global__ void __launch_bounds__(128) decode_append_kernel(
-    int64_t capacity, const int32_t* __restrict__ ctx, int B, uint16_t* __restrict__ k_idx_cache,
-    uint16_t* __restrict__ K_cache, uint16_t* __restrict__ V_cache, float* __restrict__ ksum_cache,
-    const uint16_t* __restrict__ k_idx_new, const uint16_t* __restrict__ K_new,
-    const uint16_t* __restrict__ V_new) {
-  griddep_wait();
-  griddep_launch();
-  const int64_t b = blockIdx.x;
-  const int64_t t = ctx[b];
-  if (t < 0 || t >= capacity) return;
-  const int tid = threadIdx.x;
+// The caches the append writes and the new token's rows.
+struct AppendArgs {
+  uint16_t *k_idx_cache, *K_cache, *V_cache;
+  float* ksum_cache;
+  const uint16_t *k_idx_new, *K_new, *V_new;
+  int DA;
+};
+
+// Appends sequence b's new token at position t (all threads of the CTA take
+// part) and writes the block sum of a block the token completes.
+template <int DI>
+__device__ void append_token(const AppendArgs& a, int64_t b, int64_t t, int64_t capacity, int B) {
+  const int tid = threadIdx.x, nt = blockDim.x;
   const int64_t row = b * capacity + t;
-  for (int e = tid; e < DI / 8; e += 128)
-    reinterpret_cast<uint4*>(k_idx_cache + row * DI)[e] = reinterpret_cast<const uint4*>(k_idx_new + b * DI)[e];
-  for (int e = tid; e < DA / 8; e += 128) {
-    reinterpret_cast<uint4*>(K_cache + row * DA)[e] = reinterpret_cast<const uint4*>(K_new + b * DA)[e];
-    reinterpret_cast<uint4*>(V_cache + row * DA)[e] = reinterpret_cast<const uint4*>(V_new + b * DA)[e];
+  for (int e = tid; e < DI / 8; e += nt)
+    reinterpret_cast<uint4*>(a.k_idx_cache + row * DI)[e] = reinterpret_cast<const uint4*>(a.k_idx_new + b * DI)[e];
+  for (int e = tid; e < a.DA / 8; e += nt) {
+    reinterpret_cast<uint4*>(a.K_cache + row * a.DA)[e] = reinterpret_cast<const uint4*>(a.K_new + b * a.DA)[e];
+    reinterpret_cast<uint4*>(a.V_cache + row * a.DA)[e] = reinterpret_cast<const uint4*>(a.V_new + b * a.DA)[e];
   }
   if ((t + 1) % B != 0) return;
-  // The token completes block t/B: its representative is the fp32 sum of
-  // the block's rows (the new row taken from the input, the rest from the cache).
   const int64_t blk = t / B;
-  for (int c = tid; c < DI; c += 128) {
+  for (int c = tid; c < DI; c += nt) {
     float s = 0.f;
     for (int64_t j = blk * B; j < t; ++j)
-      s += __uint_as_float(uint32_t(k_idx_cache[(b * capacity + j) * DI + c]) << 16);
-    s += __uint_as_float(uint32_t(k_idx_new[b * DI + c]) << 16);
-    ksum_cache[(b * (capacity / B) + blk) * DI + c] = s;
+      s += __uint_as_float(uint32_t(a.k_idx_cache[(b * capacity + j) * DI + c]) << 16);
+    s += __uint_as_float(uint32_t(a.k_idx_new[b * DI + c]) << 16);
+    a.ksum_cache[(b * (capacity / B) + blk) * DI + c] = s;
   }
 }
 
@@ -46,13 +49,17 @@ __global__ void __launch_bounds__(256) decode_block_scores_kernel(const int32_t*
                                                                   int B, int m, int per_cta,
                                                                   const uint16_t* __restrict__ q_new,
                                                                   const float* __restrict__ ksum_cache,
-                                                                  uint32_t* __restrict__ bkeys, int64_t ld) {
+                                                                  uint32_t* __restrict__ bkeys, int64_t ld,
+                                                                  AppendArgs ap) {
   griddep_wait();
   griddep_launch();
   constexpr int VPL = DI / 32;  // fp32 values per lane
   const int64_t b = blockIdx.x;
   const int64_t t = ctx[b];
   if (t < 0 || t >= capacity) return;
+  // the first CTA of each sequence appends the new token; the block sum it may
+  // write is the own block's, which the scores below never read
+  if (blockIdx.y == 0) append_token<DI>(ap, b, t, capacity, B);
   const int64_t nb = t / B + 1;
   if (nb <= m) return;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -145,7 +152,7 @@ __global__ void __launch_bounds__(128) decode_token_scores_kernel(const int32_t*
 // O[b][h][:] from the parts of a split query: with M the largest part
 // maximum, O = sum_p 2^(m_p - M) O_p / sum_p 2^(m_p - M) l_p (log2 units).
 // One CTA per (sequence, head), one thread per output element.
-__global__ void decode_combine_kernel(const int32_t* __restrict__ ctx, int64_t capacity, int H, int D, int parts,
+__global__ void decode_combine_kernel(int32_t* __restrict__ ctx, int64_t capacity, int H, int D, int parts,
                                       const float* __restrict__ Opart, const float* __restrict__ mpart,
                                       const float* __restrict__ lpart, uint16_t* __restrict__ O) {
   griddep_wait();
@@ -155,7 +162,6 @@ __global__ void decode_combine_kernel(const int32_t* __restrict__ ctx, int64_t c
   // every load issued before any is used: the sequence length, each part's
   // maximum, row sum and output element
   constexpr int PMAX = 16;
-  const int64_t t = ctx[b];
   float lv[PMAX], mv[PMAX], ov[PMAX];
 #pragma unroll
   for (int p = 0; p < PMAX; ++p) {
@@ -166,8 +172,9 @@ __global__ void decode_combine_kernel(const int32_t* __restrict__ ctx, int64_t c
       ov[p] = Opart[(w * H + h) * D + threadIdx.x];
     }
   }
+  // a sequence that took no step has only empty parts (row sums 0): O = 0
   float out = 0.f;
-  if (t >= 0 && t < capacity) {
+  {
     float M = -INFINITY;
 #pragma unroll
     for (int p = 0; p < PMAX; ++p)
@@ -184,22 +191,31 @@ __global__ void decode_combine_kernel(const int32_t* __restrict__ ctx, int64_t c
     out = den > 0.f ? num / den : 0.f;
   }
   O[(b * H + h) * D + threadIdx.x] = uint16_t(f32_to_bf16_rn(out));
+  // every earlier kernel of the step has finished reading the lengths: the
+  // sequence grows by one token
+  if (h == 0 && threadIdx.x == 0) {
+    const int32_t t = ctx[b];
+    if (t >= 0 && t < capacity) ctx[b] = t + 1;
+  }
 }
 
 void launch_decode_block_scores(int batch, int64_t capacity, const int32_t* ctx, int B, int m, int d_idx,
                                 const void* q_new, const float* ksum_cache, uint32_t* bkeys, int64_t ld,
-                                cudaStream_t s) {
+                                int d, void* k_idx_cache, void* K_cache, void* V_cache, float* ksum_w,
+                                const void* k_idx_new, const void* K_new, const void* V_new, cudaStream_t s) {
   if (batch == 0) return;
   const int64_t nbmax = capacity / B;
   const int per_cta = 128;
-  const dim3 grid((unsigned)batch, (unsigned)((nbmax + per_cta - 1) / per_cta));
+  const dim3 grid((unsigned)batch, (unsigned)std::max<int64_t>(1, (nbmax + per_cta - 1) / per_cta));
+  AppendArgs ap{(uint16_t*)k_idx_cache, (uint16_t*)K_cache, (uint16_t*)V_cache, ksum_w,
+                (const uint16_t*)k_idx_new, (const uint16_t*)K_new, (const uint16_t*)V_new, d};
   count_launches(1);
   if (d_idx == 128)
     launch_kernel(true, decode_block_scores_kernel<128>, grid, 256, 0, s, ctx, capacity, B, m, per_cta,
-                  (const uint16_t*)q_new, ksum_cache, bkeys, ld);
+                  (const uint16_t*)q_new, (const float*)ksum_cache, bkeys, ld, ap);
   else
     launch_kernel(true, decode_block_scores_kernel<64>, grid, 256, 0, s, ctx, capacity, B, m, per_cta,
-                  (const uint16_t*)q_new, ksum_cache, bkeys, ld);
+                  (const uint16_t*)q_new, (const float*)ksum_cache, bkeys, ld, ap);
 }
 
 void launch_decode_token_scores(int batch, int64_t capacity, const int32_t* ctx, int B, int m, int d_idx,
@@ -216,42 +232,12 @@ void launch_decode_token_scores(int batch, int64_t capacity, const int32_t* ctx,
                   (const uint16_t*)q_new, (const uint16_t*)k_idx_cache, tkeys);
 }
 
-void launch_decode_combine(int batch, int64_t capacity, const int32_t* ctx, int H, int d, int parts,
+void launch_decode_combine(int batch, int64_t capacity, int32_t* ctx, int H, int d, int parts,
                            const float* Opart, const float* mpart, const float* lpart, void* O, cudaStream_t s) {
   if (batch == 0) return;
   count_launches(1);
   launch_kernel(true, decode_combine_kernel, unsigned(batch * H), d, 0, s, ctx, capacity, H, d, parts, Opart, mpart,
                 lpart, (uint16_t*)O);
-}
-
-__global__ void decode_advance_kernel(int batch, int64_t capacity, int32_t* ctx) {
-  griddep_wait();
-  griddep_launch();
-  const int b = blockIdx.x * blockDim.x + threadIdx.x;
-  if (b < batch && ctx[b] >= 0 && ctx[b] < capacity) ctx[b] += 1;
-}
-
-void launch_decode_append(int batch, int64_t capacity, const int32_t* ctx, int B, int d_idx, int d,
-                          void* k_idx_cache, void* K_cache, void* V_cache, float* ksum_cache,
-                          const void* k_idx_new, const void* K_new, const void* V_new,
-                          cudaStream_t s) {
-  if (batch == 0) return;
-  count_launches(1);
-#define HSA_APPEND(DI, DA)                                                                      \
-  launch_kernel(true, decode_append_kernel<DI, DA>, batch, 128, 0, s, capacity, ctx, B,           \
-                (uint16_t*)k_idx_cache, (uint16_t*)K_cache, (uint16_t*)V_cache, ksum_cache,       \
-                (const uint16_t*)k_idx_new, (const uint16_t*)K_new, (const uint16_t*)V_new)
-  if (d_idx == 128 && d == 128) HSA_APPEND(128, 128);
-  else if (d_idx == 128) HSA_APPEND(128, 64);
-  else if (d == 128) HSA_APPEND(64, 128);
-  else HSA_APPEND(64, 64);
-#undef HSA_APPEND
-}
-
-void launch_decode_advance(int batch, int64_t capacity, int32_t* ctx, cudaStream_t s) {
-  if (batch == 0) return;
-  count_launches(1);
-  launch_kernel(true, decode_advance_kernel, (batch + 127) / 128, 128, 0, s, batch, capacity, ctx);
 }
 
 }  // namespace hsa

@@ -168,7 +168,7 @@ __global__ void __launch_bounds__(256) select_tokens_kernel(RowMap rm, const uin
   __shared__ uint32_t hist[RadixSelect<NT>::kBins];
   __shared__ int scratch[NT / 32 + 8];
   __shared__ float qs[D];
-  __shared__ int blk[256];
+  __shared__ int blk[512];
   __shared__ int s_nblk;
   const int64_t i = blockIdx.x;
   int32_t* out = indices + i * int64_t(k);
@@ -231,10 +231,10 @@ __global__ void __launch_bounds__(256) select_tokens_kernel(RowMap rm, const uin
 
 void launch_select_tokens(RowMap rm, int64_t rows, const void* q_idx, const void* k_idx,
                           const int32_t* blocks, int B, int m, int k, int d_idx, int32_t* indices,
-                          cudaStream_t s) {
+                          int64_t max_cand, cudaStream_t s) {
   if (rows == 0) return;
   count_launches(1);
-  const size_t smem = size_t(m) * B * 4;
+  const size_t smem = size_t(max_cand) * 4;
   if (d_idx == 128) {
     cudaFuncSetAttribute(select_tokens_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     select_tokens_kernel<128><<<unsigned(rows), 256, smem, s>>>(

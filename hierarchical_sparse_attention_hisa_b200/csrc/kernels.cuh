@@ -40,17 +40,15 @@ void launch_block_sums(const void* k_idx, int64_t Lk, int B, int d_idx, float* k
 void launch_select_blocks(RowMap rm, int64_t rows, const void* q_idx, const float* ksum,
                           int64_t ksum_seq_stride, int B, int m, int d_idx, int32_t* blocks,
                           int64_t max_cand, cudaStream_t s);
+// max_cand: the most candidates any row can have (its keys are staged in shared memory)
 void launch_select_tokens(RowMap rm, int64_t rows, const void* q_idx, const void* k_idx,
                           const int32_t* blocks, int B, int m, int k, int d_idx, int32_t* indices,
-                          cudaStream_t s);
-void launch_sparse_attn_simple(RowMap rm, int64_t rows, const void* Q, const void* K, const void* V,
-                               const int32_t* idx, int k, int H, int d, float scale, void* O,
-                               cudaStream_t s, bool pdl = false);
-// Tensor-core sparse attention (d = 128, 1 <= H <= 64); returns false if a
-// tensor map or launch attribute could not be set up.
+                          int64_t max_cand, cudaStream_t s);
+// Tensor-core sparse attention (d = 64 or 128, any H: one launch per group of
+// up to 64 heads); returns false if a launch attribute could not be set.
 bool tc_attn_supported(int H, int d, int64_t Lq, int64_t Lk);
 bool launch_sparse_attn_tc(int64_t Lq, const void* Q, const void* K, const void* V, const int32_t* idx,
-                           int64_t Lk, int k, int H, float scale, void* O, cudaStream_t s);
+                           int64_t Lk, int k, int H, int d, float scale, void* O, cudaStream_t s);
 void launch_ksum_split(const float* ksum, int64_t n, void* split, cudaStream_t s);
 bool launch_block_score_gemm(const void* q_idx, const void* bsplit, int64_t Lq, int64_t Lk, int B, int m,
                              int d_idx, int64_t nbc, uint32_t* out, int64_t ld, cudaStream_t s);
@@ -64,26 +62,28 @@ void launch_pair_lists(RowMap rm, int64_t rows, const int32_t* blocks, int B, in
                        cudaStream_t s);
 void launch_topk_from_keys(RowMap rm, int64_t rows, const int32_t* blocks, const uint32_t* tkeys, int B,
                            int m, int k, int32_t* indices, cudaStream_t s, bool pdl = false);
-void launch_decode_append(int batch, int64_t capacity, const int32_t* ctx, int B, int d_idx, int d,
-                          void* k_idx_cache, void* K_cache, void* V_cache, float* ksum_cache,
-                          const void* k_idx_new, const void* K_new, const void* V_new,
-                          cudaStream_t s);
+// (also appends each sequence's new token: k_idx/K/V rows and a completed block's sum)
 void launch_decode_block_scores(int batch, int64_t capacity, const int32_t* ctx, int B, int m, int d_idx,
                                 const void* q_new, const float* ksum_cache, uint32_t* bkeys, int64_t ld,
-                                cudaStream_t s);
+                                int d, void* k_idx_cache, void* K_cache, void* V_cache, float* ksum_w,
+                                const void* k_idx_new, const void* K_new, const void* V_new, cudaStream_t s);
 void launch_decode_token_scores(int batch, int64_t capacity, const int32_t* ctx, int B, int m, int d_idx,
                                 const int32_t* blocks, const void* q_new, const void* k_idx_cache,
                                 uint32_t* tkeys, cudaStream_t s);
-void launch_decode_combine(int batch, int64_t capacity, const int32_t* ctx, int H, int d, int parts,
+// (also advances ctx: every sequence that took the step grows by one token)
+void launch_decode_combine(int batch, int64_t capacity, int32_t* ctx, int H, int d, int parts,
                            const float* Opart, const float* mpart, const float* lpart, void* O, cudaStream_t s);
 bool launch_sparse_attn_tc_split(int batch, const void* Q, const void* Kc, const void* Vc, const int32_t* idx,
-                                 int64_t capacity, int k, int H, float scale, int parts, float* Opart,
+                                 int64_t capacity, int k, int H, int d, float scale, int parts, float* Opart,
                                  float* mpart, float* lpart, cudaStream_t s, bool pdl = false);
-void launch_decode_advance(int batch, int64_t capacity, int32_t* ctx, cudaStream_t s);
 
 // Sticky per-device flags set by a bounded wait that gave up (1), read on the
 // host with a synchronous copy and optionally cleared; -1 on a CUDA error.
 int attn_wait_flag(bool reset);
+// Test hook of the tensor-core kernels on the current device: short bounded
+// waits and one lost producer arrival in the next launch of CTA 0.
+bool attn_set_inject(bool on);
+bool score_set_inject(bool on);
 int score_wait_flag(bool reset);
 
 }  // namespace hsa

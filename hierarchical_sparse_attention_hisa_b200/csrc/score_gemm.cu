@@ -25,6 +25,9 @@
 namespace hsa {
 
 __device__ int g_score_err;
+__device__ int g_score_inject;  // test hook: short waits and one tile never produced
+
+constexpr long long kInjectWaitCycles = 1ll << 21;  // about a millisecond
 
 namespace {
 
@@ -32,7 +35,8 @@ using namespace tc;
 
 HSA_DEV bool sg_wait(uint64_t* bar, uint32_t parity, bool& dead) {
   if (dead) return false;
-  if (mbar_wait_bounded(bar, parity, &g_score_err)) return true;
+  const long long lim = *(volatile int*)&g_score_inject ? kInjectWaitCycles : kWaitCycles;
+  if (mbar_wait_bounded(bar, parity, &g_score_err, lim)) return true;
   dead = true;
   return false;
 }
@@ -136,6 +140,8 @@ __global__ void __launch_bounds__(192, 1) score_gemm_kernel(const __grid_constan
       }
       const int s = it % C::NS;
       if (!sg_wait_warp(&empty[s], ((it / C::NS) & 1) ^ 1, dead)) break;
+      // test hook: CTA 0 never produces its first tile, so its consumer's wait runs out
+      if (it == 0 && blockIdx.x == 0 && *(volatile int*)&g_score_inject) { ++it; continue; }
       uint8_t* a_s = sm + s * C::STAGE;
       uint8_t* b_s = a_s + C::A_BYTES;
       if (lane == 0) mbar_arrive_expect_tx(&full[s], C::STAGE);
@@ -291,11 +297,19 @@ bool launch_token_score_gemm(const void* q_idx, const void* k_idx, int64_t Lq, i
   if (d_idx == 128) {
     if (B == 128) return launch_sg<128, 128, 1, true>(am, bm, ta, grid, s);
     if (B == 64) return launch_sg<128, 64, 1, true>(am, bm, ta, grid, s);
+    if (B == 256) return launch_sg<128, 256, 1, true>(am, bm, ta, grid, s);
   } else {
     if (B == 128) return launch_sg<64, 128, 1, true>(am, bm, ta, grid, s);
     if (B == 64) return launch_sg<64, 64, 1, true>(am, bm, ta, grid, s);
+    if (B == 256) return launch_sg<64, 256, 1, true>(am, bm, ta, grid, s);
   }
   return false;
+}
+
+// Host side: turn the scoring kernels' test hook on or off on the current device.
+bool score_set_inject(bool on) {
+  const int v = on ? 1 : 0;
+  return cudaMemcpyToSymbol(g_score_inject, &v, sizeof v) == cudaSuccess;
 }
 
 // Host side: whether a bounded wait of this kernel gave up on the current

@@ -14,6 +14,7 @@ namespace hsa {
 namespace {
 
 constexpr int NT = 256;
+constexpr int kMaxRowBlocks = 512;  // kept blocks per row the selections hold in shared memory
 
 // Kept-block list of one row: count of valid entries and candidate count
 // (tokens j <= t of the kept blocks). Returns false when the list does not
@@ -146,7 +147,7 @@ __global__ void __launch_bounds__(NT) topk_from_keys_kernel(RowMap rm, const int
   griddep_launch();
   __shared__ uint32_t hist[RegSelect<NT, KPT>::kBins];
   __shared__ int scratch[NT / 32 + 8];
-  __shared__ int blk[256];
+  __shared__ int blk[kMaxRowBlocks];
   __shared__ int s_info[3];
   const int64_t i = blockIdx.x;
   int32_t* out = indices + i * int64_t(k);
@@ -217,11 +218,11 @@ HSA_DEV void warp_stream_keys(const uint32_t* __restrict__ row, int n, F f) {
 __global__ void __launch_bounds__(32 * kWarpRowsPerCta) topk_warp_rows_kernel(
     RowMap rm, int64_t rows, const int32_t* __restrict__ blocks, const uint32_t* __restrict__ tkeys, int B,
     int m, int k, int32_t* __restrict__ indices) {
-  extern __shared__ uint32_t wsm[];  // per warp: kWBins histogram bins, then 256 block ids
+  extern __shared__ uint32_t wsm[];  // per warp: kWBins histogram bins, then kMaxRowBlocks block ids
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t i = int64_t(blockIdx.x) * kWarpRowsPerCta + warp;
   if (i >= rows) return;
-  uint32_t* hist = wsm + warp * (kWBins + 256);
+  uint32_t* hist = wsm + warp * (kWBins + kMaxRowBlocks);
   int* blk = reinterpret_cast<int*>(hist + kWBins);
   int32_t* out = indices + i * int64_t(k);
   if (!rm.valid(i)) {
@@ -681,7 +682,7 @@ void launch_topk_from_keys(RowMap rm, int64_t rows, const int32_t* blocks, const
 #undef HSA_TOPK
   } else {
     // many longer rows: one warp per row
-    const int smem = kWarpRowsPerCta * (kWBins + 256) * 4;
+    const int smem = kWarpRowsPerCta * (kWBins + kMaxRowBlocks) * 4;
     cudaFuncSetAttribute(topk_warp_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     topk_warp_rows_kernel<<<unsigned((rows + kWarpRowsPerCta - 1) / kWarpRowsPerCta), 32 * kWarpRowsPerCta, smem,
                             s>>>(rm, rows, blocks, tkeys, B, m, k, indices);

@@ -58,17 +58,36 @@ HSA_DEV bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
 // never hang the GPU.
 constexpr long long kWaitCycles = 1ll << 32;
 constexpr uint32_t kSuspendNs = 100000;
-HSA_DEV bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* err) {
+// The same with an explicit limit in SM cycles (a test can shorten it) and a
+// suspend hint scaled to it.
+HSA_DEV bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* err, long long limit) {
   if (mbar_try_wait(bar, parity)) return true;
+  const uint32_t ns = limit < kWaitCycles ? 1000u : kSuspendNs;
   const long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
+    if (mbar_try_wait_sleep(bar, parity, ns)) return true;
     if ((it & 15u) == 0 && *(volatile int*)err) return false;
-    if (clock64() - t0 > kWaitCycles) break;
+    if (clock64() - t0 > limit) break;
   }
   atomicExch(err, 1);
   return false;
 }
+HSA_DEV bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* err) {
+  return mbar_wait_bounded(bar, parity, err, kWaitCycles);
+}
+
+// Named barrier `id` over `count` threads (a multiple of 32) that also ORs a
+// predicate across them: every participant gets the same answer.
+HSA_DEV bool bar_or(int id, int count, bool v) {
+  uint32_t out;
+  asm volatile(
+      "{\n .reg .pred a, b;\n setp.ne.u32 a, %3, 0;\n bar.red.or.pred b, %1, %2, a;\n selp.u32 %0, 1, 0, b;\n}"
+      : "=r"(out)
+      : "r"(id), "r"(count), "r"(uint32_t(v))
+      : "memory");
+  return out != 0;
+}
+HSA_DEV void bar_sync(int id, int count) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory"); }
 
 // 2^x on the special-function unit (PTX ex2.approx.ftz.f32: relative error
 // about 2^-22, subnormal results flushed to zero, 2^-inf = 0).
@@ -100,6 +119,11 @@ HSA_DEV void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar, int x
 // 16-byte global -> shared copy through the async-copy path (bypasses L1).
 HSA_DEV void cp_async16(uint32_t dst_smem, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_smem), "l"(src) : "memory");
+}
+// The same copy when `valid`, else 16 zero bytes written without reading `src`.
+HSA_DEV void cp_async16_zfill(uint32_t dst_smem, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst_smem), "l"(src), "r"(valid ? 16u : 0u)
+               : "memory");
 }
 // Arrive on `bar` once all of this thread's earlier cp.async copies land
 // (the arrival is one of the barrier's expected arrivals).
@@ -188,6 +212,37 @@ HSA_DEV void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
 }
 HSA_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 HSA_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// 32 lanes x N consecutive 32-bit columns as floats (N a multiple of 8), one wait.
+template <int N>
+HSA_DEV void tmem_load_f32(uint32_t taddr, float (&v)[N]) {
+  static_assert(N % 8 == 0, "whole 8-column groups");
+  uint32_t r[N];
+  if constexpr (N % 16 == 0) {
+#pragma unroll
+    for (int c = 0; c < N / 16; ++c) tmem_ld16(taddr + 16 * c, *reinterpret_cast<uint32_t(*)[16]>(r + 16 * c));
+  } else {
+#pragma unroll
+    for (int c = 0; c < N / 8; ++c) tmem_ld8(taddr + 8 * c, *reinterpret_cast<uint32_t(*)[8]>(r + 8 * c));
+  }
+  tmem_wait_ld();
+#pragma unroll
+  for (int e = 0; e < N; ++e) v[e] = __uint_as_float(r[e]);
+}
+template <int N>
+HSA_DEV void tmem_store_f32(uint32_t taddr, const float (&v)[N]) {
+  static_assert(N % 8 == 0, "whole 8-column groups");
+  uint32_t r[N];
+#pragma unroll
+  for (int e = 0; e < N; ++e) r[e] = __float_as_uint(v[e]);
+  if constexpr (N % 16 == 0) {
+#pragma unroll
+    for (int c = 0; c < N / 16; ++c) tmem_st16(taddr + 16 * c, *reinterpret_cast<const uint32_t(*)[16]>(r + 16 * c));
+  } else {
+#pragma unroll
+    for (int c = 0; c < N / 8; ++c) tmem_st8(taddr + 8 * c, *reinterpret_cast<const uint32_t(*)[8]>(r + 8 * c));
+  }
+  tmem_wait_st();
+}
 
 // ----------------------------------------------------------------- descriptors
 // Shared-memory matrix descriptor (sm_100 UMMA): start address, leading and

@@ -72,12 +72,14 @@ enum {
 /* Method and layer sizes. */
 typedef struct hsa_params {
   int32_t B;     /* tokens per block, 1 <= B <= 1024                           */
-  int32_t m;     /* kept blocks per query incl. the 2 forced ones, 2 <= m <= 256,
-                    m*B <= 16384 candidates                                    */
+  int32_t m;     /* kept blocks per query incl. the 2 forced ones, 2 <= m <= 512;
+                    m*B <= 65536 candidates for B in {64, 128, 256} (scored on
+                    tensor cores), m*B <= 16384 for other block sizes         */
   int32_t k;     /* kept tokens per query, 1 <= k <= 8192 (k >= m*B keeps every
                     candidate of the kept blocks)                              */
   int32_t d_idx; /* indexer head dim: 64 or 128                                 */
-  int32_t H;     /* query heads sharing one K/V head: 1 <= H <= 128             */
+  int32_t H;     /* query heads sharing one K/V head: 1 <= H <= 128 (one pass of
+                    the attention per group of up to 64 heads)                */
   int32_t d;     /* attention head dim: 64 or 128                               */
   float scale;   /* softmax scale; 0 selects 1/sqrt(d)                          */
 } hsa_params;
@@ -251,6 +253,20 @@ HSA_API uint64_t hsa_kernel_launches(void);
  * after reading them. A diagnostic for tests and benchmarks, not for the hot
  * path. */
 HSA_API int hsa_device_status(int reset);
+
+/* Test hook for the bounded-wait machinery, not for production use. The pages
+ * describe no such interface. With on != 0, on the current device: every
+ * bounded wait of the tensor-core kernels (block/token scoring, attention)
+ * gives up after about a millisecond instead of about two seconds, and the
+ * next launch of each of them loses one producer hand-off in its first CTA
+ * (the scoring kernels skip producing their first tile; the attention's first
+ * K-tile arrival is not made), so a consumer's wait must run out. The kernels
+ * then return with incomplete outputs and hsa_device_status reports
+ * HSA_ERR_TIMEOUT. Nothing faults, traps or spins without bound. With on == 0
+ * the kernels behave normally again; clear the flag with
+ * hsa_device_status(1) afterwards. Synchronous (cudaMemcpyToSymbol); returns
+ * HSA_OK, or HSA_ERR_CUDA / HSA_ERR_DEVICE. */
+HSA_API int hsa_debug_inject_lost_arrival(int on);
 
 #ifdef __cplusplus
 }

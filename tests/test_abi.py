@@ -146,7 +146,7 @@ def test_prefill_host_checks_on_the_host(lib):
 def test_device_status_without_a_gpu(lib):
     import torch
     if torch.cuda.is_available():
-        pytest.skip("a GPU is present: covered by test_zzz_wait_status")
+        pytest.skip("a GPU is present: covered by test_zz_wait_status")
     from hierarchical_sparse_attention_hisa_b200._lib import HSA_ERR_CUDA
     assert lib.hsa_device_status(0) == HSA_ERR_CUDA
 

@@ -216,6 +216,37 @@ def test_index_long_candidate_rows_bit_exact(hsa, Lq, Lk, B, m, k, seed):
     assert bad.size == 0, f"{bad.size} rows differ, first {bad[:8].tolist()}"
 
 
+@pytest.mark.parametrize("Lq,Lk,B,m,k,seed", [
+    (2000, 20000, 256, 16, 1000, 55),    # B = 256 on tensor cores
+    (500, 30000, 256, 64, 2048, 56),     # B = 256, 16,384 candidates, one warp per row
+    (100, 30000, 256, 40, 3000, 57),     # B = 256, few rows: a 1024-thread CTA per row
+    (300, 40000, 64, 512, 4096, 58),     # m = 512 (32,768 candidates), blocks pruned
+    (120, 70000, 128, 512, 2048, 59),    # m = 512 at B = 128: 65,536 candidates, few rows
+])
+def test_index_wide_rows_bit_exact(hsa, Lq, Lk, B, m, k, seed):
+    q, kk = synth.int_bf16((Lq, 128), seed, 1), synth.int_bf16((Lk, 128), seed, 2)
+    got = run_index(hsa, q, kk, B, m, k)
+    want = oracle.index(q, kk, B, m, k)
+    bad = np.flatnonzero(np.any(got != want, axis=1))
+    assert bad.size == 0, f"{bad.size} rows differ, first {bad[:8].tolist()}"
+
+
+def test_index_flat_64k_sampled(hsa):
+    # the flat token-level indexer at 64K: m = 512 keeps every causal block, so
+    # every causal token of a query is a candidate (up to 65,536 per row)
+    w = synth.WORKLOADS["prefill_64k"]
+    x = synth.prefill_inputs(w, with_attn=False)
+    m = w.L // w.B
+    got = run_index(hsa, x["q_idx"], x["k_idx"], w.B, m, w.k)
+    rows = sample_rows(w.Lq, 1024, 60, always=[0, w.k - 1, w.k, w.Lq // 2, w.Lq - 1])
+    want = oracle.index(x["q_idx"], x["k_idx"], w.B, m, w.k, rows=rows)
+    bad = np.flatnonzero(np.any(got[rows] != want, axis=1))
+    assert bad.size == 0, f"{bad.size} rows differ, first {rows[bad[:8]].tolist()}"
+    # structure of every row: ascending, causal, min(t + 1, k) valid entries
+    valid = got >= 0
+    assert (valid.sum(axis=1) == np.minimum(np.arange(w.Lq) + 1, w.k)).all()
+
+
 # ------------------------------------------------------------------ attention
 
 def test_attention_tiny_prefill_all_rows(hsa):
