@@ -68,8 +68,8 @@ __global__ void __launch_bounds__(256) decode_block_scores_kernel(const int32_t*
   for (int e = 0; e < VPL; ++e) q[e] = __uint_as_float(uint32_t(q_new[b * DI + lane * VPL + e]) << 16);
   const int64_t lo = 1 + int64_t(blockIdx.y) * per_cta, hi = min(nb - 1, lo + per_cta);
   const float* base = ksum_cache + b * (capacity / B) * DI;
-  // four block rows per warp in flight before any of them is reduced
-  constexpr int U = 4;
+  // eight block rows per warp in flight before any of them is reduced
+  constexpr int U = 8;
   for (int64_t blk0 = lo + warp; blk0 < hi; blk0 += 8 * U) {
     float v[U][VPL];
 #pragma unroll
@@ -205,7 +205,7 @@ void launch_decode_block_scores(int batch, int64_t capacity, const int32_t* ctx,
                                 const void* k_idx_new, const void* K_new, const void* V_new, cudaStream_t s) {
   if (batch == 0) return;
   const int64_t nbmax = capacity / B;
-  const int per_cta = 128;
+  const int per_cta = 64;
   const dim3 grid((unsigned)batch, (unsigned)std::max<int64_t>(1, (nbmax + per_cta - 1) / per_cta));
   AppendArgs ap{(uint16_t*)k_idx_cache, (uint16_t*)K_cache, (uint16_t*)V_cache, ksum_w,
                 (const uint16_t*)k_idx_new, (const uint16_t*)K_new, (const uint16_t*)V_new, d};

@@ -449,6 +449,12 @@ def test_decode_small_all_sequences(hsa):
                 capacity=1024, steps=70, seed=40)
 
 
+def test_decode_wide_rows(hsa):
+    # 19,200 candidates per query: the long-row top-k kernels on decode rows
+    decode_case(hsa, B=64, m=300, k=1000, d_idx=64, H=4, d=64, ctx0=[30000, 20000, 20095],
+                capacity=32768, steps=3, seed=43)
+
+
 def test_decode_128k_all_sequences(hsa):
     # the 128K decode workload's shape, every sequence checked: the contexts
     # start one token short of 1024 full blocks, so step 0 completes block
