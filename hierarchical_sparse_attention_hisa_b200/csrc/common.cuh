@@ -240,6 +240,7 @@ struct RadixSelect {
 template <int NT, int KPT>
 struct RegSelect {
   static constexpr int kBins = 2048;
+  static constexpr int kRank = 64;  // largest threshold bin ranked pairwise
   static_assert(kBins % NT == 0, "bins per thread");
   uint32_t* hist;   // smem, kBins entries
   int* scratch;     // smem, NT/32 + 8 ints
@@ -307,7 +308,33 @@ struct RegSelect {
         if (p0 + j < n) atomicAdd(&hist[vbin(key[j])], 1u);
       __syncthreads();
       const uint32_t bin = pick(rem);
-      const bool whole = hist[bin] == uint32_t(rem);
+      const uint32_t cstar = hist[bin];
+      const bool whole = cstar == uint32_t(rem);
+      if (!whole && cstar <= uint32_t(kRank)) {
+        // a bin of at most kRank keys: gather it and rank it pairwise, the
+        // rem-th largest of the bin is T
+        if (threadIdx.x == 0) s[4] = 0;
+        __syncthreads();  // (hist[bin] has been read by every thread)
+#pragma unroll
+        for (int j = 0; j < KPT; ++j)
+          if (p0 + j < n && vbin(key[j]) == bin) hist[atomicAdd((int*)&s[4], 1)] = key[j];
+        __syncthreads();
+        if (threadIdx.x < int(cstar)) {
+          const uint32_t x = hist[threadIdx.x];
+          int gt = 0, ge = 0;
+          for (int q = 0; q < int(cstar); ++q) {
+            const uint32_t y = hist[q];
+            gt += y > x;
+            ge += y >= x;
+          }
+          if (gt < rem && rem <= ge) { s[0] = int(x); s[1] = rem - gt; }  // writers agree
+        }
+        __syncthreads();
+        *T_out = uint32_t(s[0]);
+        *take_eq = s[1];
+        __syncthreads();  // s[] is read before any later use of the scratch
+        return;
+      }
       key_range([&](uint32_t u) { return vbin(u) == bin; }, &base, &kmax);
       if (whole && base > 0u) {
         *T_out = base - 1u;

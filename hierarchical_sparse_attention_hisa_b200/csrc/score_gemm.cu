@@ -9,16 +9,19 @@
 //                  bf16 MMAs accumulate the fp32 result;
 //   token scores   S[i][s][c] = q_idx[i] . k_idx[b*B + c]   for every (query i,
 //                  slot s) that kept block b: queries that kept the same block
-//                  are gathered (TMA tile::gather4) as the 128 rows of one MMA
-//                  tile against that block's B keys, so each key block is read
-//                  once per 128 queries instead of once per query.
+//                  are gathered (cp.async, one 16-byte piece per lane) as the
+//                  128 rows of one MMA tile against that block's B keys, so
+//                  each key block is read once per 128 queries instead of
+//                  once per query.
 // Integer-valued inputs make every product and partial sum an exact fp32
 // integer, so the tensor-core results equal the sequential CPU sums.
 //
-// Warp roles of the persistent kernel: warp 0 TMA producer, warp 1 MMA issuer
-// (+ TMEM owner), warps 2-5 epilogue (TMEM -> keys -> global), with a
-// two-deep TMEM accumulator so the epilogue of one tile overlaps the MMAs of
-// the next.
+// Warp roles of the persistent kernel: warp 0 TMA producer (the B tiles, and
+// the A tiles of block scoring), warp 1 MMA issuer (+ TMEM owner), warps 2-5
+// epilogue (TMEM -> keys -> global through a shared-memory staging tile),
+// and for token scoring warps 6-9, which copy the gathered query rows. The
+// TMEM accumulator is two deep, so the epilogue of one tile overlaps the MMAs
+// of the next.
 #include "kernels.cuh"
 #include "tc.cuh"
 
@@ -67,6 +70,7 @@ struct TileArgs {
   const int* ntiles;        // device count of tiles
   const uint32_t* pairs;    // pair = row * m + slot
   int m, Bsz;
+  const void* qsrc;         // gathered mode: q_idx rows [Lq][DK] bf16
   // tiled mode (block scores)
   int Lq, Lk, nb_tiles, m_tiles, nbc;
   // output
@@ -83,8 +87,11 @@ HSA_DEV bool block_tile_needed(const TileArgs& a, int mt, int nt, int N) {
   return int64_t(nt) * N <= nb_last - 2;       // candidates are blocks 1 .. nb-2
 }
 
+// gathered mode: 4 more warps copy the query rows with cp.async
+template <bool GATHER> constexpr int sg_threads() { return GATHER ? 320 : 192; }
+
 template <int DK, int N, int NSPLIT, bool GATHER>
-__global__ void __launch_bounds__(192, 1) score_gemm_kernel(const __grid_constant__ CUtensorMap amap,
+__global__ void __launch_bounds__(sg_threads<GATHER>(), 1) score_gemm_kernel(const __grid_constant__ CUtensorMap amap,
                                                             const __grid_constant__ CUtensorMap bmap,
                                                             TileArgs ta) {
   using C = SG<DK, N, NSPLIT>;
@@ -92,9 +99,11 @@ __global__ void __launch_bounds__(192, 1) score_gemm_kernel(const __grid_constan
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ __align__(8) uint64_t full[C::NS], empty[C::NS], tfull[2], tempty[2], done;
   __shared__ uint32_t tmem_base;
+  __shared__ __align__(16) uint32_t stage[4][32 * 32];  // epilogue staging, one tile per warp
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::NS; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    // gathered mode: the TMA bytes of B plus one arrival per query-row copying thread
+    for (int s = 0; s < C::NS; ++s) { mbar_init(&full[s], GATHER ? 1 + 128 : 1); mbar_init(&empty[s], 1); }
     for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], 4); }
     mbar_init(&done, 1);
     fence_barrier_init();
@@ -111,27 +120,13 @@ __global__ void __launch_bounds__(192, 1) score_gemm_kernel(const __grid_constan
     // ------------------------------------------------------------ producer
     if (lane == 0) { prefetch_tmap(&amap); prefetch_tmap(&bmap); }
     uint32_t it = 0;
-    // a gathered tile's descriptor and query rows take two dependent global
-    // loads: they are fetched one tile ahead
-    int4 dn = make_int4(0, 0, 0, 0);
-    int rn[4] = {0, 0, 0, 0};
-    auto fetch = [&](int tt) {
-      if (tt >= total) return;
-      dn = ta.tiles[tt];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int r = lane * 4 + e;
-        rn[e] = r < dn.z ? int(ta.pairs[dn.y + r] / uint32_t(ta.m)) : 0;
-      }
-    };
-    if (GATHER) fetch(blockIdx.x);
+    // a gathered tile's descriptor (its key block) is fetched one tile ahead
+    int bn = (GATHER && blockIdx.x < total) ? ta.tiles[blockIdx.x].x : 0;
     for (int t = blockIdx.x; t < total && !dead; t += gridDim.x) {
-      int a_row0 = 0, b_row0 = 0, rows[4] = {0, 0, 0, 0};
+      int a_row0 = 0, b_row0 = 0;
       if (GATHER) {
-        b_row0 = dn.x * ta.Bsz;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) rows[e] = rn[e];
-        fetch(t + gridDim.x);
+        b_row0 = bn * ta.Bsz;
+        if (t + int(gridDim.x) < total) bn = ta.tiles[t + gridDim.x].x;
       } else {
         const int mt = t / ta.nb_tiles, nt = t % ta.nb_tiles;
         if (!block_tile_needed(ta, mt, nt, N)) continue;
@@ -144,13 +139,9 @@ __global__ void __launch_bounds__(192, 1) score_gemm_kernel(const __grid_constan
       if (it == 0 && blockIdx.x == 0 && *(volatile int*)&g_score_inject) { ++it; continue; }
       uint8_t* a_s = sm + s * C::STAGE;
       uint8_t* b_s = a_s + C::A_BYTES;
-      if (lane == 0) mbar_arrive_expect_tx(&full[s], C::STAGE);
+      if (lane == 0) mbar_arrive_expect_tx(&full[s], GATHER ? C::B_BYTES : C::STAGE);
       __syncwarp();
-      if (GATHER) {
-#pragma unroll
-        for (int kb = 0; kb < C::KB; ++kb)
-          tma_gather4(a_s + kb * 128 * 128 + lane * 512, &amap, &full[s], kb * 64, rows[0], rows[1], rows[2], rows[3]);
-      } else if (lane == 0) {
+      if (!GATHER && lane == 0) {
 #pragma unroll
         for (int kb = 0; kb < C::KB; ++kb) tma_load_2d(a_s + kb * 128 * 128, &amap, &full[s], kb * 64, a_row0);
       }
@@ -180,6 +171,7 @@ __global__ void __launch_bounds__(192, 1) score_gemm_kernel(const __grid_constan
         if (!sg_wait(&full[s], (it / C::NS) & 1, dead)) break;
         if (!sg_wait(&tempty[tb], ((it >> 1) & 1) ^ 1, dead)) break;
         tc_fence_after();
+        if (GATHER) fence_proxy_async_smem();  // query rows landed by cp.async, read by the MMA
         const uint32_t a_s = smem_u32(sm + s * C::STAGE);
         const uint32_t b_s = a_s + C::A_BYTES;
         uint32_t acc = 0;
@@ -201,36 +193,84 @@ __global__ void __launch_bounds__(192, 1) score_gemm_kernel(const __grid_constan
       sg_wait(&done, 0, d2);
     }
     __syncwarp();
+  } else if (GATHER && warp >= 6) {
+    // ------------------------------------------------------------ query-row copies
+    // warp 6 + g copies rows 32g .. 32g+31 of each tile: lane l fetches the
+    // query row of tile row 32g + l, the copying lanes take it by shuffle
+    constexpr int CPR = DK / 8;          // 16-byte chunks per row
+    constexpr int RPI = 32 / CPR;        // rows per warp instruction
+    const int gw = warp - 6, c = lane % CPR, rsub = lane / CPR;
+    const uint4* qb = reinterpret_cast<const uint4*>(ta.qsrc);
+    uint32_t it = 0;
+    auto qrow_of = [&](int tt) -> int {
+      if (tt >= total) return 0;
+      const int4 d = ta.tiles[tt];
+      const int r = 32 * gw + lane;
+      return r < d.z ? int(ta.pairs[d.y + r] / uint32_t(ta.m)) : 0;
+    };
+    int qn = qrow_of(blockIdx.x);
+    for (int t = blockIdx.x; t < total && !dead; t += gridDim.x) {
+      const int qr = qn;
+      qn = qrow_of(t + gridDim.x);  // one tile ahead
+      const int s = it % C::NS;
+      if (!sg_wait_warp(&empty[s], ((it / C::NS) & 1) ^ 1, dead)) break;
+      const uint32_t a_s = smem_u32(sm + s * C::STAGE);
+#pragma unroll
+      for (int u = 0; u < 32 / RPI; ++u) {
+        const int rr = u * RPI + rsub, row = 32 * gw + rr;
+        const int q = __shfl_sync(kFull, qr, rr);
+        cp_async16(a_s + (c >> 3) * (128 * 128) + row * 128 + (((c & 7) ^ (row & 7)) << 4),
+                   qb + int64_t(q) * CPR + c);
+      }
+      cp_async_arrive(&full[s]);
+      ++it;
+    }
+    cp_async_wait_all();  // every copy has landed before the CTA may exit
   } else {
     // ------------------------------------------------------------ epilogue
+    // Each warp owns 32 accumulator rows (its TMEM lane quarter). Keys go out
+    // 32 columns at a time through a 32 x 128-byte staging tile (16-byte
+    // chunks XOR-swizzled by row), so that every global store instruction
+    // writes four whole 128-byte row segments instead of 32 scattered pieces.
     const int quad = warp & 3, r = quad * 32 + lane;
     const uint32_t lane_addr = uint32_t(quad * 32) << 16;
+    uint32_t* sb = stage[quad];
+    const int rsub = lane >> 3, ch = lane & 7;
     uint32_t it = 0;
     for (int t = blockIdx.x; t < total && !dead; t += gridDim.x) {
-      uint32_t* dst = nullptr;
+      int64_t off = -1;  // element offset of this thread's row in out, or -1
       if (GATHER) {
         const int4 d = ta.tiles[t];
-        if (r < d.z) dst = ta.out + int64_t(ta.pairs[d.y + r]) * ta.ld;
+        if (r < d.z) off = int64_t(ta.pairs[d.y + r]) * ta.ld;
       } else {
         const int mt = t / ta.nb_tiles, nt = t % ta.nb_tiles;
         if (!block_tile_needed(ta, mt, nt, N)) continue;
         const int row = mt * 128 + r;
-        if (row < ta.Lq) dst = ta.out + int64_t(row) * ta.ld + int64_t(nt) * N;
+        if (row < ta.Lq) off = int64_t(row) * ta.ld + int64_t(nt) * N;
       }
+      // the rows this thread stores: 4 * i + rsub of the warp's 32
+      int64_t roff[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) roff[i] = __shfl_sync(kFull, off, 4 * i + rsub);
       const int tb = it & 1;
       if (!sg_wait_warp(&tfull[tb], (it >> 1) & 1, dead)) break;
       tc_fence_after();
-#pragma unroll 2
-      for (int c0 = 0; c0 < N; c0 += 16) {
-        uint32_t v[16];
-        tmem_ld16(tmem + lane_addr + tb * N + c0, v);
-        tmem_wait_ld();
-        if (dst) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+#pragma unroll 1
+      for (int c0 = 0; c0 < N; c0 += 32) {
+        float v[32];
+        tmem_load_f32<32>(tmem + lane_addr + tb * N + c0, v);
+        __syncwarp();  // the previous chunk has been read out of the staging tile
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            d4[e] = make_uint4(score_key(__uint_as_float(v[4 * e])), score_key(__uint_as_float(v[4 * e + 1])),
-                               score_key(__uint_as_float(v[4 * e + 2])), score_key(__uint_as_float(v[4 * e + 3])));
+        for (int e = 0; e < 8; ++e)
+          *reinterpret_cast<uint4*>(sb + lane * 32 + ((e ^ (lane & 7)) << 2)) =
+              make_uint4(score_key(v[4 * e]), score_key(v[4 * e + 1]), score_key(v[4 * e + 2]),
+                         score_key(v[4 * e + 3]));
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int rr = 4 * i + rsub;
+          const uint4 x = *reinterpret_cast<const uint4*>(sb + rr * 32 + ((ch ^ (rr & 7)) << 2));
+          if (roff[i] >= 0) *reinterpret_cast<uint4*>(ta.out + roff[i] + c0 + 4 * ch) = x;
         }
       }
       tc_fence_before();
@@ -252,7 +292,7 @@ bool launch_sg(const CUtensorMap& am, const CUtensorMap& bm, const TileArgs& ta,
   using C = SG<DK, N, NSPLIT>;
   auto kern = score_gemm_kernel<DK, N, NSPLIT, GATHER>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess) return false;
-  kern<<<grid, 192, C::SMEM, s>>>(am, bm, ta);
+  kern<<<grid, sg_threads<GATHER>(), C::SMEM, s>>>(am, bm, ta);
   count_launches(1);
   return true;
 }
@@ -286,12 +326,13 @@ bool launch_block_score_gemm(const void* q_idx, const void* bsplit, int64_t Lq, 
 bool launch_token_score_gemm(const void* q_idx, const void* k_idx, int64_t Lq, int64_t Lk, int B, int m,
                              int d_idx, const int4* tiles, const int* ntiles, const uint32_t* pairs,
                              int64_t max_tiles, uint32_t* out, cudaStream_t s) {
-  CUtensorMap am, bm;
-  if (!make_tmap_2d(&am, q_idx, uint64_t(Lq), uint64_t(d_idx), 1) ||
-      !make_tmap_2d(&bm, k_idx, uint64_t(Lk), uint64_t(d_idx), B))
-    return false;
+  // the query rows are copied by cp.async: only the key blocks go through a tensor map
+  (void)Lq;
+  CUtensorMap bm;
+  if (!make_tmap_2d(&bm, k_idx, uint64_t(Lk), uint64_t(d_idx), B)) return false;
+  const CUtensorMap& am = bm;
   TileArgs ta{};
-  ta.tiles = tiles; ta.ntiles = ntiles; ta.pairs = pairs; ta.m = m; ta.Bsz = B;
+  ta.tiles = tiles; ta.ntiles = ntiles; ta.pairs = pairs; ta.m = m; ta.Bsz = B; ta.qsrc = q_idx;
   ta.out = out; ta.ld = B;
   const int grid = int(max_tiles < num_sms() ? (max_tiles > 0 ? max_tiles : 1) : num_sms());
   if (d_idx == 128) {

@@ -30,6 +30,25 @@ HSA_DEV bool row_candidates(const int32_t* blk, int m, int64_t t, int B, int* nb
   return true;
 }
 
+// The same check by the 32 lanes of a warp together (every lane gets the
+// result): lane l reads entries l, l + 32, ... of the list.
+HSA_DEV bool warp_row_candidates(const int32_t* blk, int m, int64_t t, int B, int* nblk_out, int* ncand_out) {
+  const int lane = threadIdx.x & 31;
+  int nblk = m;
+  for (int s0 = 0; s0 < m && nblk == m; s0 += 32) {
+    const int s = s0 + lane;
+    const unsigned neg = __ballot_sync(kFull, s < m && blk[s] < 0);
+    if (neg) nblk = s0 + __ffs(neg) - 1;
+  }
+  if (nblk == 0) return false;  // (warp-uniform)
+  bool ok = true;
+  for (int s = lane; s + 1 < nblk; s += 32) ok = ok && blk[s] < blk[s + 1];
+  ok = __all_sync(kFull, ok) && blk[nblk - 1] == int(t / B);
+  *nblk_out = nblk;
+  *ncand_out = int((nblk - 1) * int64_t(B) + (t - int64_t(blk[nblk - 1]) * B + 1));
+  return ok;
+}
+
 template <int KPT>
 __global__ void __launch_bounds__(NT) topm_from_keys_kernel(RowMap rm, const uint32_t* __restrict__ bkeys,
                                                            int64_t ld, int B, int m, int32_t* __restrict__ blocks) {
@@ -64,6 +83,74 @@ __global__ void __launch_bounds__(NT) topm_from_keys_kernel(RowMap rm, const uin
   rs.compact(key, n, T, take_eq, [&](int rank, int c) { out[1 + rank] = c + 1; });
 }
 
+// Top-m with one warp per row, for rows of at most 32 * KPT candidate blocks
+// (many rows, few candidates each: no CTA barriers). Lane l holds the keys of
+// candidates e * 32 + l. The threshold T, the (m-2)-th largest key, is built
+// bit by bit from the top: a bit is kept when at least m - 2 keys are >= the
+// value with it set. Selected candidates are written in ascending order, ties
+// at T going to the lowest positions, exactly as the block-wide selection.
+constexpr int kTopmWarpsPerCta = 8;
+
+template <int KPT>
+__global__ void __launch_bounds__(32 * kTopmWarpsPerCta) topm_warp_rows_kernel(
+    RowMap rm, int64_t rows, const uint32_t* __restrict__ bkeys, int64_t ld, int B, int m,
+    int32_t* __restrict__ blocks) {
+  griddep_wait();
+  griddep_launch();
+  const int lane = threadIdx.x & 31;
+  const int64_t i = int64_t(blockIdx.x) * kTopmWarpsPerCta + (threadIdx.x >> 5);
+  if (i >= rows) return;
+  int32_t* out = blocks + i * m;
+  if (!rm.valid(i)) {
+    for (int s = lane; s < m; s += 32) out[s] = -1;
+    return;
+  }
+  const int64_t t = rm.pos(i);
+  const int64_t nb = t / B + 1;
+  if (nb <= m) {
+    for (int s = lane; s < m; s += 32) out[s] = s < nb ? s : -1;
+    return;
+  }
+  if (m == 2) {
+    if (lane == 0) { out[0] = 0; out[1] = int32_t(nb - 1); }
+    return;
+  }
+  const int n = int(nb - 2);  // candidates: blocks 1 .. nb-2
+  const int r = m - 2;
+  const uint32_t* src = bkeys + i * ld + 1;
+  uint32_t key[KPT];
+#pragma unroll
+  for (int e = 0; e < KPT; ++e) key[e] = e * 32 + lane < n ? __ldg(src + e * 32 + lane) : 0u;
+  // count of this lane's keys >= x (keys past n never count)
+  auto count_ge = [&](uint32_t x) {
+    int c = 0;
+#pragma unroll
+    for (int e = 0; e < KPT; ++e) c += (e * 32 + lane < n && key[e] >= x) ? 1 : 0;
+    return __reduce_add_sync(kFull, c);
+  };
+  uint32_t T = 0;
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t c = T | (1u << bit);
+    if (count_ge(c) >= r) T = c;
+  }
+  const int take_eq = T == 0xffffffffu ? r : r - count_ge(T + 1);
+  if (lane == 0) { out[0] = 0; out[m - 1] = int32_t(nb - 1); }
+  const unsigned below = (1u << lane) - 1u;
+  int base = 0, eqb = 0;
+#pragma unroll
+  for (int e = 0; e < KPT; ++e) {
+    const int c = e * 32 + lane;
+    const bool live = c < n;
+    const bool gt = live && key[e] > T, eq = live && key[e] == T;
+    const unsigned beq = __ballot_sync(kFull, eq);
+    const bool take = gt || (eq && eqb + __popc(beq & below) < take_eq);
+    const unsigned bt = __ballot_sync(kFull, take);
+    if (take) out[1 + base + __popc(bt & below)] = c + 1;
+    base += __popc(bt);
+    eqb += __popc(beq);
+  }
+}
+
 // Pairs of the rows [r0, r0 + ROWS) that need token scores, binned by block.
 constexpr int kPairRows = 64;
 
@@ -87,7 +174,7 @@ __global__ void __launch_bounds__(NT) pair_bin_kernel(RowMap rm, int64_t rows, c
       const int32_t* blk = blocks + i * m;
       const int64_t t = rm.pos(i);
       int nblk = 0, ncand = 0;
-      if (!row_candidates(blk, m, t, B, &nblk, &ncand) || ncand <= k) continue;
+      if (!warp_row_candidates(blk, m, t, B, &nblk, &ncand) || ncand <= k) continue;
       for (int s = lane; s < nblk; s += 32) fn(i, s, blk[s]);
     }
   };
@@ -233,7 +320,7 @@ __global__ void __launch_bounds__(32 * kWarpRowsPerCta) topk_warp_rows_kernel(
   for (int s = lane; s < m; s += 32) blk[s] = blocks[i * m + s];
   __syncwarp();
   int nblk = 0, n = 0;
-  const bool ok = row_candidates(blk, m, t, B, &nblk, &n);
+  const bool ok = warp_row_candidates(blk, m, t, B, &nblk, &n);
   if (!ok) {
     for (int s = lane; s < k; s += 32) out[s] = -1;
     return;
@@ -642,6 +729,17 @@ void launch_topm_from_keys(RowMap rm, int64_t rows, const uint32_t* bkeys, int64
                            int64_t max_cand, int32_t* blocks, cudaStream_t s, bool pdl) {
   if (rows == 0) return;
   count_launches(1);
+  if (max_cand <= 512 && rows >= 8 * int64_t(num_sms())) {
+    // many rows of few candidates: one warp per row
+    const unsigned grid = unsigned((rows + kTopmWarpsPerCta - 1) / kTopmWarpsPerCta);
+    if (max_cand <= 256)
+      launch_kernel(pdl, topm_warp_rows_kernel<8>, grid, 32 * kTopmWarpsPerCta, 0, s, rm, rows, bkeys, ld, B, m,
+                    blocks);
+    else
+      launch_kernel(pdl, topm_warp_rows_kernel<16>, grid, 32 * kTopmWarpsPerCta, 0, s, rm, rows, bkeys, ld, B, m,
+                    blocks);
+    return;
+  }
 #define HSA_TOPM(K) launch_kernel(pdl, topm_from_keys_kernel<K>, unsigned(rows), NT, 0, s, rm, bkeys, ld, B, m, blocks)
   HSA_KPT_DISPATCH(keys_per_thread(max_cand), HSA_TOPM)
 #undef HSA_TOPM

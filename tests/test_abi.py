@@ -94,7 +94,7 @@ def test_workspace_sizes_on_host(lib):
 
 
 @pytest.mark.parametrize("field,value", [("B", 0), ("m", 1), ("k", 0), ("d_idx", 96),
-                                         ("m", 300), ("B", 2048)])
+                                         ("m", 513), ("B", 2048)])
 def test_bad_index_params_rejected(lib, field, value):
     import hierarchical_sparse_attention_hisa_b200 as hsa
     p = hsa.params(B=128, m=64, k=2048, d_idx=128)
@@ -103,6 +103,16 @@ def test_bad_index_params_rejected(lib, field, value):
     assert lib.hsa_index_workspace_size(ctypes.byref(p), 100, 200, ctypes.byref(n)) == 1
     # the full call is rejected on the host as well (no pointers needed)
     assert lib.hsa_index(ctypes.byref(p), 100, 200, None, None, None, None, 0, None) == 1
+
+
+@pytest.mark.parametrize("B,m,ok", [(128, 512, True), (256, 256, True), (256, 257, False),
+                                    (96, 170, True), (96, 171, False)])
+def test_candidate_limits(lib, B, m, ok):
+    # at most 65,536 candidates per row (m * B) when B is 64, 128 or 256, else 16,384
+    import hierarchical_sparse_attention_hisa_b200 as hsa
+    p = hsa.params(B=B, m=m, k=256, d_idx=128)
+    n = ctypes.c_size_t(0)
+    assert (lib.hsa_index_workspace_size(ctypes.byref(p), 100, 200, ctypes.byref(n)) == 0) == ok
 
 
 def test_bad_lengths_and_pointers_rejected(lib):
