@@ -429,10 +429,11 @@ __global__ void __launch_bounds__(32 * kWarpRowsPerCta) topk_warp_rows_kernel(
 // chunk of each of its threads are both free of bank conflicts.
 // The threshold is located first in 2048 bins linear in the score value
 // (bins on key bits would crowd a row into the few bins of its exponent
-// range). A value bin is a contiguous key range, found exactly by bisection
-// of the bin function, and usually holds a handful of keys, which are
+// range). The bin function never decreases as the score grows, so a bin is a
+// contiguous key range; it usually holds a handful of keys, which are
 // gathered and ranked directly. A crowded bin, or a row whose score range is
-// not finite, continues with 11-bit rounds on the key bits.
+// not finite, continues with 11-bit rounds on the key bits. The k selected
+// indices are assembled in shared memory and leave with coalesced stores.
 constexpr int kRowNT = 256, kRowCap = 8192, kRowKPT = kRowCap / kRowNT, kRowChunks = kRowKPT / 4;
 constexpr int kRowBins = 2048, kRowBPT = kRowBins / kRowNT;
 constexpr int kRowRank = 64;  // largest threshold bin ranked pairwise
@@ -507,6 +508,7 @@ __global__ void __launch_bounds__(kRowNT, 4) topk_rows_kernel(RowMap rm, const i
   }
   const int p0 = tid * kRowKPT;
   const int nj = max(0, min(kRowKPT, n - p0));  // this thread's candidates: keys j < nj
+  const uint32_t jmask = nj >= 32 ? 0xffffffffu : (1u << nj) - 1u;
   auto chunk = [&](int c) { return S.keys[(tid << 3) | (c ^ (tid & 7))]; };
   auto key_at = [&](int j) {
     const uint4 v = chunk(j >> 2);
@@ -573,10 +575,18 @@ __global__ void __launch_bounds__(kRowNT, 4) topk_rows_kernel(RowMap rm, const i
 
   uint32_t ulo, uhi;
   {
+    // this thread's key range (keys past nj stand in as the other bound)
     uint32_t lo = 0xffffffffu, hi = 0u;
-    each([&](int j, uint32_t u) {
-      if (j < nj) { lo = min(lo, u); hi = max(hi, u); }
-    });
+#pragma unroll
+    for (int c = 0; c < kRowChunks; ++c) {
+      const uint4 v = chunk(c);
+      const uint32_t a0 = 4 * c < nj ? v.x : 0xffffffffu, a1 = 4 * c + 1 < nj ? v.y : 0xffffffffu;
+      const uint32_t a2 = 4 * c + 2 < nj ? v.z : 0xffffffffu, a3 = 4 * c + 3 < nj ? v.w : 0xffffffffu;
+      const uint32_t b0 = 4 * c < nj ? v.x : 0u, b1 = 4 * c + 1 < nj ? v.y : 0u;
+      const uint32_t b2 = 4 * c + 2 < nj ? v.z : 0u, b3 = 4 * c + 3 < nj ? v.w : 0u;
+      lo = __vimin3_u32(lo, a0, __vimin3_u32(a1, a2, a3));
+      hi = __vimax3_u32(hi, b0, __vimax3_u32(b1, b2, b3));
+    }
     block_min_max(lo, hi, &ulo, &uhi);
   }
   int rem = k;
@@ -587,29 +597,35 @@ __global__ void __launch_bounds__(kRowNT, 4) topk_rows_kernel(RowMap rm, const i
   const float flo = key_score(ulo), fhi = key_score(uhi);
   const float c = float(kRowBins) / (fhi - flo);
   if (flo < fhi && c > 0.f && c < INFINITY) {
-    // the bin fma(x, c, -lo * c), rounded to nearest and truncated, never
-    // decreases as x grows
-    const float nb = -flo * c;
+    // the bin of score x: (x - lo) * c rounded to an integer by adding
+    // 1.5 * 2^23 in one fma and reading the low bits of the sum (the sum stays
+    // positive, and positive float bit patterns grow with the value, so the
+    // bin never decreases as x grows), clamped to [0, kRowBins)
+    const float nb = 12582912.0f - flo * c;
     uint32_t vbr[kRowKPT / 2];  // the bins of keys 2r and 2r + 1
 #pragma unroll
     for (int r = 0; r < kRowKPT / 2; ++r) vbr[r] = 0;
     each([&](int j, uint32_t u) {
-      const uint32_t b = min(uint32_t(kRowBins - 1), __float2uint_rz(fmaf(key_score(u), c, nb)));
+      const int bi = int(__float_as_uint(fmaf(key_score(u), c, nb)) - 0x4B400000u);
+      const uint32_t b = uint32_t(min(kRowBins - 1, max(0, bi)));
       if (j < nj) atomicAdd(&S.hist[b], 1u);
       vbr[j >> 1] |= b << (16 * (j & 1));
     });
     __syncthreads();
     const uint32_t bin = pick(rem);
     const uint32_t cstar = S.hist[bin];
-    uint32_t binm = 0;  // this thread's keys inside the bin
+    // keys in bins above the threshold bin, and keys inside it (two per
+    // packed 16-bit comparison)
+    const uint32_t bin2 = bin | (bin << 16);
+    uint32_t binm = 0;
 #pragma unroll
-    for (int j = 0; j < kRowKPT; ++j) {
-      const uint32_t b = (vbr[j >> 1] >> (16 * (j & 1))) & 0xffffu;
-      if (j < nj) {
-        gtm |= uint32_t(b > bin) << j;
-        binm |= uint32_t(b == bin) << j;
-      }
+    for (int r = 0; r < kRowKPT / 2; ++r) {
+      const uint32_t g2 = __vcmpgtu2(vbr[r], bin2), e2 = __vcmpeq2(vbr[r], bin2);
+      gtm |= ((g2 & 1u) | ((g2 >> 15) & 2u)) << (2 * r);
+      binm |= ((e2 & 1u) | ((e2 >> 15) & 2u)) << (2 * r);
     }
+    gtm &= jmask;
+    binm &= jmask;
     if (cstar <= uint32_t(kRowRank)) {
       // gather the bin and rank it pairwise: T is its rem-th largest key
       for (uint32_t mm = binm; mm; mm &= mm - 1u) S.list[atomicAdd(&S.red[16], 1u)] = key_at(__ffs(mm) - 1);
@@ -691,17 +707,32 @@ __global__ void __launch_bounds__(kRowNT, 4) topk_rows_kernel(RowMap rm, const i
 #pragma unroll
   for (int u = 0; u < kRowNT / 32; ++u)
     if (u < w) before += S.sc[8 + u];
-  int G = before >> 16, Q = before & 0xffff;
-  for (uint32_t mm = gtm | eqm; mm; mm &= mm - 1u) {
-    const int j = __ffs(mm) - 1;
-    const int32_t tk = (S.blk[(p0 + j) >> lb] << lb) + ((p0 + j) & (B - 1));
-    if ((gtm >> j) & 1u) {
-      out[G + min(Q, take_eq)] = tk;
-      ++G;
-    } else {
-      if (Q < take_eq) out[G + Q] = tk;
-      ++Q;
+  const int G = before >> 16, Q = before & 0xffff;
+  // the keys equal to T that are taken: the first take_eq - Q of this thread's
+  uint32_t sel = gtm;
+  for (uint32_t mm = eqm, q = uint32_t(Q); mm && q < uint32_t(take_eq); mm &= mm - 1u, ++q) sel |= mm & (0u - mm);
+  // The row's k indices are assembled in shared memory (over the keys, which
+  // every thread has finished reading: the barrier above) and then written
+  // out with coalesced stores. This thread's 32 positions lie in one kept
+  // block when B >= 32; its selected tokens are then tok0 + j, in
+  // consecutive slots.
+  int32_t* so = reinterpret_cast<int32_t*>(S.keys);
+  int32_t* o = so + G + min(Q, take_eq);
+  if (B >= kRowKPT) {
+    const int32_t tok0 = (S.blk[p0 >> lb] << lb) + (p0 & (B - 1));
+    for (uint32_t mm = sel; mm; mm &= mm - 1u) *o++ = tok0 + (__ffs(mm) - 1);
+  } else {
+    for (uint32_t mm = sel; mm; mm &= mm - 1u) {
+      const int p = p0 + __ffs(mm) - 1;
+      *o++ = (S.blk[p >> lb] << lb) + (p & (B - 1));
     }
+  }
+  __syncthreads();
+  if ((k & 3) == 0 && (reinterpret_cast<uintptr_t>(out) & 15u) == 0) {
+    for (int e = tid; e < k / 4; e += kRowNT)
+      reinterpret_cast<int4*>(out)[e] = reinterpret_cast<const int4*>(so)[e];
+  } else {
+    for (int e = tid; e < k; e += kRowNT) out[e] = so[e];
   }
 }
 
