@@ -28,7 +28,8 @@
 // only raised (and O^T, l rescaled) when a tile exceeds it by more than 2^8,
 // so the cross-thread max reduction happens on a query's first tile and
 // rarely after; the per-tile check is one hardware barrier reduction. P is
-// rounded to bf16 for the second MMA; accumulation is fp32.
+// rounded to bf16 for the second MMA; accumulation is fp32; O is normalised
+// by one reciprocal of the row sum per head.
 //
 // A barrier probe in an MMA-issuing thread costs about as much as an MMA when
 // MMAs are queued, so with two stages each issuer waits on one barrier per
@@ -277,6 +278,7 @@ __global__ void __launch_bounds__(32 * Cfg<HP, DH>::NWARPS, 1) sparse_attn_tc_ke
   __shared__ float red[4][HP];
   __shared__ float mh[HP];
   __shared__ float lsum[HP];
+  __shared__ float linv[HP];  // 1 / lsum (0 where lsum is 0)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nh = a.nh;
@@ -635,7 +637,11 @@ __global__ void __launch_bounds__(32 * Cfg<HP, DH>::NWARPS, 1) sparse_attn_tc_ke
         for (int e = 0; e < NL; ++e) red[wq][h0 + transpose_head<HH>(lane, e)] = lp[e];
       }
       wg_sync(bar_id);
-      if (r < HH) lsum[h0 + r] = red[0][h0 + r] + red[1][h0 + r] + red[2][h0 + r] + red[3][h0 + r];
+      if (r < HH) {
+        const float l = red[0][h0 + r] + red[1][h0 + r] + red[2][h0 + r] + red[3][h0 + r];
+        lsum[h0 + r] = l;
+        linv[h0 + r] = l > 0.f ? 1.f / l : 0.f;
+      }
       wg_sync(bar_id);
       const bool oko = wait_all(&bars.ofull[ob], (oq >> 1) & 1, dead);
       if (oko) {
@@ -645,10 +651,7 @@ __global__ void __launch_bounds__(32 * Cfg<HP, DH>::NWARPS, 1) sparse_attn_tc_ke
         if (orow) {
 #pragma unroll
           for (int h = 0; h < HH; ++h) {
-            if (h0 + h < nh && r < DH) {
-              const float l = lsum[h0 + h];
-              orow[(h0 + h) * DH + r] = uint16_t(f32_to_bf16_rn(l > 0.f ? ov[h] / l : 0.f));
-            }
+            if (h0 + h < nh && r < DH) orow[(h0 + h) * DH + r] = uint16_t(f32_to_bf16_rn(ov[h] * linv[h0 + h]));
           }
         } else {
           // one part of a split query: unnormalised O^T, running maximum, row sum
