@@ -550,7 +550,8 @@ __global__ void __launch_bounds__(32 * Cfg<HP, DH>::NWARPS, 1) sparse_attn_tc_ke
         }
         const bool mine = tmax > kRescaleThreshold || !complete;
         dead = dead || !oks;
-        if (wg_or(bar_id, i == 0 || mine || dead)) {
+        // (a query's first tile always sets the maxima: no vote needed)
+        if (i == 0 || wg_or(bar_id, mine || dead)) {
           if (wg_or(bar_id, dead)) { quit = true; break; }
           // raise the running maxima of this warpgroup's heads to cover the tile
 #pragma unroll
@@ -599,7 +600,9 @@ __global__ void __launch_bounds__(32 * Cfg<HP, DH>::NWARPS, 1) sparse_attn_tc_ke
               tmem_st_cols<HH>(ta, ov);
             }
           }
-          wg_sync(bar_id);  // red[0] holds the old maxima until everyone has read them
+          // red[0] holds the old maxima until everyone has read them (a first
+          // tile reads none: it rescales nothing)
+          if (i > 0) wg_sync(bar_id);
         }
         // probabilities, partial row sums, this warpgroup's part of the P^T row
         const int pb = g & 1;
