@@ -1,9 +1,11 @@
 // hsa_prefill_host: the whole path (index, then sparse attention) for queries
 // whose inputs and outputs live in host memory, with the host<->device copies
-// overlapped with the kernels. The query rows are cut into chunks; while the
-// attention of chunk c runs, chunk c+1's Q rows come in and chunk c-1's O and
-// index rows go out, on two copy streams of the library's own that fork from
-// the caller's stream and join back into it.
+// overlapped with the kernels. The indices go out as soon as the indexer is
+// done; the query rows are cut into chunks, and while the attention of chunk
+// c runs, chunk c+1's Q rows come in and chunk c-1's O rows go out, on two
+// copy streams of the library's own that fork from the caller's stream and
+// join back into it. (The device-to-host direction, O and the indices, is the
+// larger: starting it with the indices keeps it busy from the indexer on.)
 #include <algorithm>
 #include <mutex>
 
@@ -21,7 +23,7 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 // device's first call and kept until the process exits.
 struct CopyStreams {
   cudaStream_t h2d = nullptr, d2h = nullptr;
-  cudaEvent_t start = nullptr, joined = nullptr;
+  cudaEvent_t start = nullptr, joined = nullptr, idx_ready = nullptr;
   cudaEvent_t q_ready[kMaxChunks] = {}, o_ready[kMaxChunks] = {};
   std::mutex mu;  // one call at a time enqueues on them
   bool ok = false;
@@ -39,7 +41,8 @@ CopyStreams* copy_streams() {
     bool good = cudaStreamCreateWithFlags(&c.h2d, cudaStreamNonBlocking) == cudaSuccess &&
                 cudaStreamCreateWithFlags(&c.d2h, cudaStreamNonBlocking) == cudaSuccess &&
                 cudaEventCreateWithFlags(&c.start, f) == cudaSuccess &&
-                cudaEventCreateWithFlags(&c.joined, f) == cudaSuccess;
+                cudaEventCreateWithFlags(&c.joined, f) == cudaSuccess &&
+                cudaEventCreateWithFlags(&c.idx_ready, f) == cudaSuccess;
     for (int i = 0; good && i < kMaxChunks; ++i)
       good = cudaEventCreateWithFlags(&c.q_ready[i], f) == cudaSuccess &&
              cudaEventCreateWithFlags(&c.o_ready[i], f) == cudaSuccess;
@@ -130,6 +133,12 @@ int hsa_prefill_host(const hsa_params* p, int64_t Lq, int64_t Lk, const hsa_bf16
     cu(cudaMemcpyAsync(k_idx, k_idx_h, size_t(Lk) * p->d_idx * 2, cudaMemcpyHostToDevice, stream));
     cu(cudaMemcpyAsync(q_idx, q_idx_h, size_t(Lq) * p->d_idx * 2, cudaMemcpyHostToDevice, stream));
     if (ok) status = hsa_index(p, Lq, Lk, q_idx, k_idx, idx, ws + w.index_ws, w.index_ws_bytes, stream);
+    // the indices out on the D2H stream, while the attention runs
+    if (ok && status == HSA_OK && indices_h) {
+      cu(cudaEventRecord(cs->idx_ready, stream));
+      cu(cudaStreamWaitEvent(cs->d2h, cs->idx_ready, 0));
+      cu(cudaMemcpyAsync(indices_h, idx, size_t(Lq) * p->k * 4, cudaMemcpyDeviceToHost, cs->d2h));
+    }
   }
   if (ok && status == HSA_OK) {
     // the attention's inputs on the H2D stream: K and V, then Q chunk by chunk
@@ -153,16 +162,13 @@ int hsa_prefill_host(const hsa_params* p, int64_t Lq, int64_t Lk, const hsa_bf16
     }
   }
   if (ok && status == HSA_OK) {
-    // each chunk's results out on the D2H stream as soon as its attention is done
+    // each chunk's O rows out on the D2H stream as soon as its attention is done
     for (int c = 0; c < n; ++c) {
       int64_t r0, rows;
       chunk_rows(Lq, n, c, &r0, &rows);
       cu(cudaStreamWaitEvent(cs->d2h, cs->o_ready[c], 0));
       cu(cudaMemcpyAsync(O_h + r0 * qrow, O + r0 * qrow, size_t(rows) * qrow * 2, cudaMemcpyDeviceToHost,
                          cs->d2h));
-      if (indices_h)
-        cu(cudaMemcpyAsync(indices_h + r0 * p->k, idx + r0 * p->k, size_t(rows) * p->k * 4,
-                           cudaMemcpyDeviceToHost, cs->d2h));
     }
   }
   // join, after a failure too: the caller's stream goes on only once every

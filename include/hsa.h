@@ -156,8 +156,9 @@ HSA_API int hsa_prefill_host_workspace_size(const hsa_params* p, int64_t Lq, int
  * streams of the library (created on a device's first call, which must not
  * be made during stream capture, and kept until the process exits) fork from
  * `stream` and join back into it: the indexer runs on `stream` while the Q
- * rows come in, the attention of a chunk starts once its Q rows have landed,
- * and a chunk's O and index rows go back while the next chunk is computed.
+ * rows come in, the indices go back as soon as the indexer is done, the
+ * attention of a chunk starts once its Q rows have landed, and a chunk's O
+ * rows go back while the next chunk is computed.
  * All of it is ordered after earlier work on `stream`, and later work on
  * `stream` runs after the last copy; the call returns once everything is
  * enqueued (synchronise `stream` before reading O_h). The copies overlap the
