@@ -49,6 +49,30 @@ HSA_DEV bool warp_row_candidates(const int32_t* blk, int m, int64_t t, int B, in
   return ok;
 }
 
+// Keys of positions [p0, p0 + KPT) of the row that starts one key after
+// `row` (p0 = threadIdx.x * KPT), positions >= n read as 0: from 16-byte
+// loads of `row` itself (aligned) shifted by one key, where the row (of ld
+// keys) holds them all, else one key at a time.
+template <int KPT>
+HSA_DEV void load_keys_after_first(const uint32_t* __restrict__ row, int64_t ld, int n, uint32_t (&key)[KPT]) {
+  const int p0 = threadIdx.x * KPT;
+  if constexpr (KPT % 4 == 0) {
+    if (p0 + KPT <= n && p0 + KPT + 4 <= ld && (reinterpret_cast<uintptr_t>(row) & 15u) == 0) {
+      uint32_t v[KPT + 4];
+#pragma unroll
+      for (int q = 0; q < KPT / 4 + 1; ++q) {
+        const uint4 x = __ldg(reinterpret_cast<const uint4*>(row + p0) + q);
+        v[4 * q] = x.x; v[4 * q + 1] = x.y; v[4 * q + 2] = x.z; v[4 * q + 3] = x.w;
+      }
+#pragma unroll
+      for (int j = 0; j < KPT; ++j) key[j] = v[j + 1];
+      return;
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) key[j] = p0 + j < n ? __ldg(row + 1 + p0 + j) : 0u;
+}
+
 template <int KPT>
 __global__ void __launch_bounds__(NT) topm_from_keys_kernel(RowMap rm, const uint32_t* __restrict__ bkeys,
                                                            int64_t ld, int B, int m, int32_t* __restrict__ blocks) {
@@ -74,7 +98,7 @@ __global__ void __launch_bounds__(NT) topm_from_keys_kernel(RowMap rm, const uin
   }
   const int n = int(nb - 2);  // candidates: blocks 1 .. nb-2
   uint32_t key[KPT];
-  load_keys<KPT>(bkeys + i * ld + 1, n, key);
+  load_keys_after_first<KPT>(bkeys + i * ld, ld, n, key);
   RegSelect<NT, KPT> rs{hist, scratch};
   uint32_t T;
   int take_eq;
