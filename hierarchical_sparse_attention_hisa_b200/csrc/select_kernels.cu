@@ -74,7 +74,7 @@ HSA_DEV void load_keys_after_first(const uint32_t* __restrict__ row, int64_t ld,
 }
 
 template <int KPT>
-__global__ void __launch_bounds__(NT) topm_from_keys_kernel(RowMap rm, const uint32_t* __restrict__ bkeys,
+__global__ void __launch_bounds__(NT, 3) topm_from_keys_kernel(RowMap rm, const uint32_t* __restrict__ bkeys,
                                                            int64_t ld, int B, int m, int32_t* __restrict__ blocks) {
   griddep_wait();
   griddep_launch();
@@ -475,7 +475,7 @@ struct RowSmem {
 
 HSA_DEV int row_slot(int g) { return (g & ~7) | ((g & 7) ^ ((g >> 3) & 7)); }
 
-__global__ void __launch_bounds__(kRowNT, 4) topk_rows_kernel(RowMap rm, const int32_t* __restrict__ blocks,
+__global__ void __launch_bounds__(kRowNT, 5) topk_rows_kernel(RowMap rm, const int32_t* __restrict__ blocks,
                                                            const uint32_t* __restrict__ tkeys, int B, int m,
                                                            int k, int32_t* __restrict__ indices) {
   griddep_wait();
