@@ -109,10 +109,10 @@ __global__ void __launch_bounds__(NT, 3) topm_from_keys_kernel(RowMap rm, const 
 
 // Top-m with one warp per row, for rows of at most 32 * KPT candidate blocks
 // (many rows, few candidates each: no CTA barriers). Lane l holds the keys of
-// candidates e * 32 + l. The threshold T, the (m-2)-th largest key, is built
-// bit by bit from the top: a bit is kept when at least m - 2 keys are >= the
-// value with it set. Selected candidates are written in ascending order, ties
-// at T going to the lowest positions, exactly as the block-wide selection.
+// candidates e * 32 + l. The threshold T, the (m-2)-th largest key, is found
+// by radix selection, 8 key bits a pass from the top, in a warp-private
+// histogram. Selected candidates are written in ascending order, ties at T
+// going to the lowest positions, exactly as the block-wide selection.
 constexpr int kTopmWarpsPerCta = 8;
 
 template <int KPT>
@@ -145,19 +145,54 @@ __global__ void __launch_bounds__(32 * kTopmWarpsPerCta) topm_warp_rows_kernel(
   uint32_t key[KPT];
 #pragma unroll
   for (int e = 0; e < KPT; ++e) key[e] = e * 32 + lane < n ? __ldg(src + e * 32 + lane) : 0u;
-  // count of this lane's keys >= x (keys past n never count)
-  auto count_ge = [&](uint32_t x) {
-    int c = 0;
+  // the (m-2)-th largest key T by radix selection on the key bits, 8 bits a
+  // pass from the top, with a warp-private 256-bin histogram (lanes holding
+  // the same digit add once, through a match)
+  __shared__ __align__(16) uint32_t whist[kTopmWarpsPerCta][256];
+  uint32_t* hist = whist[threadIdx.x >> 5];
+  uint32_t T = 0, tmask = 0;
+  int rem = r;  // rank of T among the keys that share the digits chosen so far
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    reinterpret_cast<uint4*>(hist)[2 * lane] = make_uint4(0, 0, 0, 0);
+    reinterpret_cast<uint4*>(hist)[2 * lane + 1] = make_uint4(0, 0, 0, 0);
+    __syncwarp();
 #pragma unroll
-    for (int e = 0; e < KPT; ++e) c += (e * 32 + lane < n && key[e] >= x) ? 1 : 0;
-    return __reduce_add_sync(kFull, c);
-  };
-  uint32_t T = 0;
-  for (int bit = 31; bit >= 0; --bit) {
-    const uint32_t c = T | (1u << bit);
-    if (count_ge(c) >= r) T = c;
+    for (int e = 0; e < KPT; ++e) {
+      const bool in = e * 32 + lane < n && (key[e] & tmask) == T;
+      const uint32_t d = in ? (key[e] >> shift) & 255u : 256u;
+      const unsigned same = __match_any_sync(kFull, d);
+      if (in && lane == __ffs(same) - 1) atomicAdd(&hist[d], uint32_t(__popc(same)));
+    }
+    __syncwarp();
+    // lane l holds bins 8l .. 8l+7; the keys in the bins of the lanes above
+    uint32_t cnt[8], tot = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) { cnt[q] = hist[lane * 8 + q]; tot += cnt[q]; }
+    uint32_t suf = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_down_sync(kFull, suf, o);
+      if (lane + o < 32) suf += y;
+    }
+    const uint32_t above = suf - tot;
+    const bool holds = above < uint32_t(rem) && uint32_t(rem) <= above + tot;
+    int dsel = 0, nrem = 0;
+    if (holds) {
+      uint32_t acc = above;
+#pragma unroll
+      for (int q = 7; q >= 0; --q) {
+        if (dsel == 0 && nrem == 0 && acc + cnt[q] >= uint32_t(rem)) { dsel = lane * 8 + q; nrem = rem - int(acc); }
+        acc += cnt[q];
+      }
+    }
+    const int from = __ffs(__ballot_sync(kFull, holds)) - 1;
+    dsel = __shfl_sync(kFull, dsel, from);
+    rem = __shfl_sync(kFull, nrem, from);
+    T |= uint32_t(dsel) << shift;
+    tmask |= 255u << shift;
+    __syncwarp();  // every lane has read the histogram before it is cleared
   }
-  const int take_eq = T == 0xffffffffu ? r : r - count_ge(T + 1);
+  const int take_eq = rem;
   if (lane == 0) { out[0] = 0; out[m - 1] = int32_t(nb - 1); }
   const unsigned below = (1u << lane) - 1u;
   int base = 0, eqb = 0;
