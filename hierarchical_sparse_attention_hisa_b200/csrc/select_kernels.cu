@@ -508,6 +508,19 @@ struct RowSmem {
   int pk[2];
 };
 
+// Bits 0..15 of x to the even positions, bits 16..31 to the odd ones.
+HSA_DEV uint32_t interleave_halves(uint32_t x) {
+  uint32_t t = (x ^ (x >> 8)) & 0x0000ff00u;
+  x ^= t ^ (t << 8);
+  t = (x ^ (x >> 4)) & 0x00f000f0u;
+  x ^= t ^ (t << 4);
+  t = (x ^ (x >> 2)) & 0x0c0c0c0cu;
+  x ^= t ^ (t << 2);
+  t = (x ^ (x >> 1)) & 0x22222222u;
+  x ^= t ^ (t << 1);
+  return x;
+}
+
 HSA_DEV int row_slot(int g) { return (g & ~7) | ((g & 7) ^ ((g >> 3) & 7)); }
 
 __global__ void __launch_bounds__(kRowNT, 5) topk_rows_kernel(RowMap rm, const int32_t* __restrict__ blocks,
@@ -528,9 +541,14 @@ __global__ void __launch_bounds__(kRowNT, 5) topk_rows_kernel(RowMap rm, const i
   // stage the row's key slots first (every candidate and the unused tail);
   // warp 0 checks the kept-block list while they land
   {
+    // slot g = tid + kRowNT * u lands at row_slot(tid) + kRowNT * u (the
+    // swizzle only mixes bits below kRowNT)
     const int nslot4 = (m * B) >> 2;
-    const uint4* src = reinterpret_cast<const uint4*>(tkeys + i * int64_t(m) * B);
-    for (int g = tid; g < nslot4; g += kRowNT) tc::cp_async16(tc::smem_u32(&S.keys[row_slot(g)]), src + g);
+    const uint4* src = reinterpret_cast<const uint4*>(tkeys + i * int64_t(m) * B) + tid;
+    const uint32_t dst = tc::smem_u32(&S.keys[row_slot(tid)]);
+#pragma unroll
+    for (int u = 0; u < kRowCap / 4 / kRowNT; ++u)
+      if (tid + u * kRowNT < nslot4) tc::cp_async16(dst + u * kRowNT * 16, src + u * kRowNT);
   }
   for (int e = 0; e < kRowBPT; ++e) S.hist[tid * kRowBPT + e] = 0;
   if (w == 0) {
@@ -636,15 +654,24 @@ __global__ void __launch_bounds__(kRowNT, 5) topk_rows_kernel(RowMap rm, const i
   {
     // this thread's key range (keys past nj stand in as the other bound)
     uint32_t lo = 0xffffffffu, hi = 0u;
+    if (nj == kRowKPT) {
 #pragma unroll
-    for (int c = 0; c < kRowChunks; ++c) {
-      const uint4 v = chunk(c);
-      const uint32_t a0 = 4 * c < nj ? v.x : 0xffffffffu, a1 = 4 * c + 1 < nj ? v.y : 0xffffffffu;
-      const uint32_t a2 = 4 * c + 2 < nj ? v.z : 0xffffffffu, a3 = 4 * c + 3 < nj ? v.w : 0xffffffffu;
-      const uint32_t b0 = 4 * c < nj ? v.x : 0u, b1 = 4 * c + 1 < nj ? v.y : 0u;
-      const uint32_t b2 = 4 * c + 2 < nj ? v.z : 0u, b3 = 4 * c + 3 < nj ? v.w : 0u;
-      lo = __vimin3_u32(lo, a0, __vimin3_u32(a1, a2, a3));
-      hi = __vimax3_u32(hi, b0, __vimax3_u32(b1, b2, b3));
+      for (int c = 0; c < kRowChunks; ++c) {
+        const uint4 v = chunk(c);
+        lo = __vimin3_u32(lo, v.x, __vimin3_u32(v.y, v.z, v.w));
+        hi = __vimax3_u32(hi, v.x, __vimax3_u32(v.y, v.z, v.w));
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < kRowChunks; ++c) {
+        const uint4 v = chunk(c);
+        const uint32_t a0 = 4 * c < nj ? v.x : 0xffffffffu, a1 = 4 * c + 1 < nj ? v.y : 0xffffffffu;
+        const uint32_t a2 = 4 * c + 2 < nj ? v.z : 0xffffffffu, a3 = 4 * c + 3 < nj ? v.w : 0xffffffffu;
+        const uint32_t b0 = 4 * c < nj ? v.x : 0u, b1 = 4 * c + 1 < nj ? v.y : 0u;
+        const uint32_t b2 = 4 * c + 2 < nj ? v.z : 0u, b3 = 4 * c + 3 < nj ? v.w : 0u;
+        lo = __vimin3_u32(lo, a0, __vimin3_u32(a1, a2, a3));
+        hi = __vimax3_u32(hi, b0, __vimax3_u32(b1, b2, b3));
+      }
     }
     block_min_max(lo, hi, &ulo, &uhi);
   }
@@ -654,37 +681,66 @@ __global__ void __launch_bounds__(kRowNT, 5) topk_rows_kernel(RowMap rm, const i
   uint32_t gtm = 0, eqm = 0;  // this thread's keys above T, and equal to T (bit j: key j)
   bool done = false;
   const float flo = key_score(ulo), fhi = key_score(uhi);
-  const float c = float(kRowBins) / (fhi - flo);
+  const float c = float(kRowBins - 3) / (fhi - flo);
   if (flo < fhi && c > 0.f && c < INFINITY) {
-    // the bin of score x: (x - lo) * c rounded to an integer by adding
+    // the bin of score x: (x - lo) * c + 1 rounded to an integer by adding
     // 1.5 * 2^23 in one fma and reading the low bits of the sum (the sum stays
     // positive, and positive float bit patterns grow with the value, so the
-    // bin never decreases as x grows), clamped to [0, kRowBins)
-    const float nb = 12582912.0f - flo * c;
+    // bin never decreases as x grows). When the row's smallest and largest
+    // keys land in [0, kRowBins), every key does; otherwise bins are clamped.
+    const float nb = 12582913.0f - flo * c;
     uint32_t vbr[kRowKPT / 2];  // the bins of keys 2r and 2r + 1
+    const int blo = int(__float_as_uint(fmaf(flo, c, nb)) - 0x4B400000u);
+    const int bhi = int(__float_as_uint(fmaf(fhi, c, nb)) - 0x4B400000u);
+    if (blo >= 0 && bhi < kRowBins) {
+      // the slots past this thread's candidates read as the row's smallest
+      // key (so every thread takes the same path), and the smallest key's
+      // bin gives those kRowCap - n counts back
+      for (int j = nj; j < kRowKPT; ++j)
+        reinterpret_cast<uint32_t*>(&S.keys[(tid << 3) | ((j >> 2) ^ (tid & 7))])[j & 3] = ulo;
+      if (tid == 0) atomicSub(&S.hist[blo], uint32_t(kRowCap - n));
 #pragma unroll
-    for (int r = 0; r < kRowKPT / 2; ++r) vbr[r] = 0;
-    each([&](int j, uint32_t u) {
-      const int bi = int(__float_as_uint(fmaf(key_score(u), c, nb)) - 0x4B400000u);
-      const uint32_t b = uint32_t(min(kRowBins - 1, max(0, bi)));
-      if (j < nj) atomicAdd(&S.hist[b], 1u);
-      vbr[j >> 1] |= b << (16 * (j & 1));
-    });
+      for (int cc = 0; cc < kRowChunks; ++cc) {
+        const uint4 v = chunk(cc);
+        const uint32_t b0 = __float_as_uint(fmaf(key_score(v.x), c, nb)) - 0x4B400000u;
+        const uint32_t b1 = __float_as_uint(fmaf(key_score(v.y), c, nb)) - 0x4B400000u;
+        const uint32_t b2 = __float_as_uint(fmaf(key_score(v.z), c, nb)) - 0x4B400000u;
+        const uint32_t b3 = __float_as_uint(fmaf(key_score(v.w), c, nb)) - 0x4B400000u;
+        atomicAdd(&S.hist[b0], 1u);
+        atomicAdd(&S.hist[b1], 1u);
+        atomicAdd(&S.hist[b2], 1u);
+        atomicAdd(&S.hist[b3], 1u);
+        vbr[2 * cc] = __byte_perm(b0, b1, 0x5410);
+        vbr[2 * cc + 1] = __byte_perm(b2, b3, 0x5410);
+      }
+    } else {
+#pragma unroll
+      for (int r = 0; r < kRowKPT / 2; ++r) vbr[r] = 0;
+      each([&](int j, uint32_t u) {
+        const int bi = int(__float_as_uint(fmaf(key_score(u), c, nb)) - 0x4B400000u);
+        const uint32_t b = uint32_t(min(kRowBins - 1, max(0, bi)));
+        if (j < nj) atomicAdd(&S.hist[b], 1u);
+        vbr[j >> 1] |= b << (16 * (j & 1));
+      });
+    }
     __syncthreads();
     const uint32_t bin = pick(rem);
     const uint32_t cstar = S.hist[bin];
-    // keys in bins above the threshold bin, and keys inside it (two per
-    // packed 16-bit comparison)
-    const uint32_t bin2 = bin | (bin << 16);
-    uint32_t binm = 0;
+    // keys in bins above the threshold bin, and keys inside it, two per
+    // subtraction: with bit 15 of each 11-bit half set, subtracting bin + 1
+    // (bin) from both halves leaves bit 15 set exactly where the half's bin is
+    // above (at least) the threshold bin; the flags of keys 2r and 2r + 1 are
+    // collected in bits r and 16 + r, then interleaved into key order
+    const uint32_t above2 = (bin + 1u) * 0x10001u, atleast2 = bin * 0x10001u;
+    uint32_t gtp = 0, gep = 0;
 #pragma unroll
     for (int r = 0; r < kRowKPT / 2; ++r) {
-      const uint32_t g2 = __vcmpgtu2(vbr[r], bin2), e2 = __vcmpeq2(vbr[r], bin2);
-      gtm |= ((g2 & 1u) | ((g2 >> 15) & 2u)) << (2 * r);
-      binm |= ((e2 & 1u) | ((e2 >> 15) & 2u)) << (2 * r);
+      const uint32_t x = vbr[r] | 0x80008000u;
+      gtp |= ((x - above2) >> (15 - r)) & (0x10001u << r);
+      gep |= ((x - atleast2) >> (15 - r)) & (0x10001u << r);
     }
-    gtm &= jmask;
-    binm &= jmask;
+    gtm = interleave_halves(gtp) & jmask;
+    uint32_t binm = interleave_halves(gep & ~gtp) & jmask;
     if (cstar <= uint32_t(kRowRank)) {
       // gather the bin and rank it pairwise: T is its rem-th largest key
       for (uint32_t mm = binm; mm; mm &= mm - 1u) S.list[atomicAdd(&S.red[16], 1u)] = key_at(__ffs(mm) - 1);
