@@ -110,9 +110,11 @@ __global__ void __launch_bounds__(NT, 3) topm_from_keys_kernel(RowMap rm, const 
 // Top-m with one warp per row, for rows of at most 32 * KPT candidate blocks
 // (many rows, few candidates each: no CTA barriers). Lane l holds the keys of
 // candidates e * 32 + l. The threshold T, the (m-2)-th largest key, is found
-// by radix selection, 8 key bits a pass from the top, in a warp-private
-// histogram. Selected candidates are written in ascending order, ties at T
-// going to the lowest positions, exactly as the block-wide selection.
+// in a warp-private histogram: one pass over bins linear in the score and a
+// direct ranking of the threshold bin's keys, or, when that bin is crowded,
+// radix selection 8 key bits a pass from the top. Selected candidates are
+// written in ascending order, ties at T going to the lowest positions,
+// exactly as the block-wide selection.
 constexpr int kTopmWarpsPerCta = 8;
 
 template <int KPT>
@@ -145,26 +147,16 @@ __global__ void __launch_bounds__(32 * kTopmWarpsPerCta) topm_warp_rows_kernel(
   uint32_t key[KPT];
 #pragma unroll
   for (int e = 0; e < KPT; ++e) key[e] = e * 32 + lane < n ? __ldg(src + e * 32 + lane) : 0u;
-  // the (m-2)-th largest key T by radix selection on the key bits, 8 bits a
-  // pass from the top, with a warp-private 256-bin histogram (lanes holding
-  // the same digit add once, through a match)
   __shared__ __align__(16) uint32_t whist[kTopmWarpsPerCta][256];
+  __shared__ uint32_t wlist[kTopmWarpsPerCta][32];
   uint32_t* hist = whist[threadIdx.x >> 5];
-  uint32_t T = 0, tmask = 0;
-  int rem = r;  // rank of T among the keys that share the digits chosen so far
-  for (int shift = 24; shift >= 0; shift -= 8) {
+  auto clear_hist = [&]() {
     reinterpret_cast<uint4*>(hist)[2 * lane] = make_uint4(0, 0, 0, 0);
     reinterpret_cast<uint4*>(hist)[2 * lane + 1] = make_uint4(0, 0, 0, 0);
-    __syncwarp();
-#pragma unroll
-    for (int e = 0; e < KPT; ++e) {
-      const bool in = e * 32 + lane < n && (key[e] & tmask) == T;
-      const uint32_t d = in ? (key[e] >> shift) & 255u : 256u;
-      const unsigned same = __match_any_sync(kFull, d);
-      if (in && lane == __ffs(same) - 1) atomicAdd(&hist[d], uint32_t(__popc(same)));
-    }
-    __syncwarp();
-    // lane l holds bins 8l .. 8l+7; the keys in the bins of the lanes above
+  };
+  // the bin of the histogram holding the rem-th largest counted key; rem
+  // becomes the rank inside it (lane l holds bins 8l .. 8l+7)
+  auto pick = [&](int& rem) -> int {
     uint32_t cnt[8], tot = 0;
 #pragma unroll
     for (int q = 0; q < 8; ++q) { cnt[q] = hist[lane * 8 + q]; tot += cnt[q]; }
@@ -186,13 +178,85 @@ __global__ void __launch_bounds__(32 * kTopmWarpsPerCta) topm_warp_rows_kernel(
       }
     }
     const int from = __ffs(__ballot_sync(kFull, holds)) - 1;
-    dsel = __shfl_sync(kFull, dsel, from);
     rem = __shfl_sync(kFull, nrem, from);
-    T |= uint32_t(dsel) << shift;
-    tmask |= 255u << shift;
-    __syncwarp();  // every lane has read the histogram before it is cleared
+    return __shfl_sync(kFull, dsel, from);
+  };
+  // The (m-2)-th largest key T. First in 256 bins linear in the score (see
+  // the top-k rows): the threshold bin usually holds a few keys, which are
+  // ranked directly. Otherwise radix selection on the key bits, 8 bits a pass
+  // from the top (lanes holding the same digit add once, through a match).
+  uint32_t T = 0;
+  int take_eq = -1;
+  {
+    uint32_t lo = 0xffffffffu, hi = 0u;
+#pragma unroll
+    for (int e = 0; e < KPT; ++e)
+      if (e * 32 + lane < n) { lo = min(lo, key[e]); hi = max(hi, key[e]); }
+    lo = __reduce_min_sync(kFull, lo);
+    hi = __reduce_max_sync(kFull, hi);
+    const float flo = key_score(lo), fhi = key_score(hi);
+    const float c = 253.0f / (fhi - flo);
+    if (flo < fhi && c > 0.f && c < INFINITY) {
+      const float nb = 12582913.0f - flo * c;  // bin = (x - lo) * c + 1, rounded
+      auto bin_of = [&](uint32_t u) {
+        return min(255, max(0, int(__float_as_uint(fmaf(key_score(u), c, nb)) - 0x4B400000u)));
+      };
+      clear_hist();
+      __syncwarp();
+#pragma unroll
+      for (int e = 0; e < KPT; ++e)
+        if (e * 32 + lane < n) atomicAdd(&hist[bin_of(key[e])], 1u);
+      __syncwarp();
+      int rem = r;
+      const int bsel = pick(rem);
+      const uint32_t cstar = hist[bsel];
+      if (cstar <= 32u) {
+        // gather the threshold bin and rank its keys pairwise
+        int cnt = 0;
+#pragma unroll
+        for (int e = 0; e < KPT; ++e) {
+          const bool in = e * 32 + lane < n && bin_of(key[e]) == bsel;
+          const unsigned bi = __ballot_sync(kFull, in);
+          if (in) wlist[threadIdx.x >> 5][cnt + __popc(bi & ((1u << lane) - 1u))] = key[e];
+          cnt += __popc(bi);
+        }
+        __syncwarp();
+        int gt = 0, ge = 0;
+        const uint32_t x = lane < int(cstar) ? wlist[threadIdx.x >> 5][lane] : 0u;
+        for (int q = 0; q < int(cstar); ++q) {
+          const uint32_t y = wlist[threadIdx.x >> 5][q];
+          gt += y > x;
+          ge += y >= x;
+        }
+        const bool hit = lane < int(cstar) && gt < rem && rem <= ge;
+        const int from = __ffs(__ballot_sync(kFull, hit)) - 1;
+        T = __shfl_sync(kFull, x, from);
+        take_eq = __shfl_sync(kFull, rem - gt, from);
+      }
+      __syncwarp();  // every lane has read the histogram before it is cleared
+    }
   }
-  const int take_eq = rem;
+  if (take_eq < 0) {
+    uint32_t tmask = 0;
+    int rem = r;  // rank of T among the keys that share the digits chosen so far
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      clear_hist();
+      __syncwarp();
+#pragma unroll
+      for (int e = 0; e < KPT; ++e) {
+        const bool in = e * 32 + lane < n && (key[e] & tmask) == T;
+        const uint32_t d = in ? (key[e] >> shift) & 255u : 256u;
+        const unsigned same = __match_any_sync(kFull, d);
+        if (in && lane == __ffs(same) - 1) atomicAdd(&hist[d], uint32_t(__popc(same)));
+      }
+      __syncwarp();
+      const int dsel = pick(rem);
+      T |= uint32_t(dsel) << shift;
+      tmask |= 255u << shift;
+      __syncwarp();  // every lane has read the histogram before it is cleared
+    }
+    take_eq = rem;
+  }
   if (lane == 0) { out[0] = 0; out[m - 1] = int32_t(nb - 1); }
   const unsigned below = (1u << lane) - 1u;
   int base = 0, eqb = 0;
