@@ -91,7 +91,8 @@ int64_t max_block_candidates(const hsa_params* p, int64_t Lk) {
 //   bsplit [3][nbc][d_idx] bf16       hi/mid/lo planes of ksum
 //   bkeys  [Lq][ldb] u32              block-score keys (ldb = nbc rounded to 64)
 //   blocks [Lq][m] i32                kept blocks
-//   cnt/off/cursor [nbins] i32        pairs per key block (nbins = ceil(Lk/B))
+//   cnt/cursor [nbins] i32            pairs per key block (nbins = ceil(Lk/B))
+//   off [2][nbins] i32                first pair and first tile of each key block
 //   ntiles i32, tiles [max_tiles] int4, pairs [Lq*m] u32
 //   tkeys  [Lq][m][B] u32             token-score keys
 struct IndexWs {
@@ -111,7 +112,7 @@ IndexWs index_ws(const hsa_params* p, int64_t Lq, int64_t Lk) {
   w.bkeys = take(size_t(Lq) * w.ldb * 4);
   w.blocks = take(size_t(Lq) * p->m * 4);
   w.cnt = take(size_t(w.nbins) * 4);
-  w.off = take(size_t(w.nbins) * 4);
+  w.off = take(size_t(w.nbins) * 8);
   w.cursor = take(size_t(w.nbins) * 4);
   w.ntiles = take(16);
   w.tiles = take(size_t(w.max_tiles) * 16);

@@ -275,13 +275,15 @@ __global__ void __launch_bounds__(32 * kTopmWarpsPerCta) topm_warp_rows_kernel(
 }
 
 // Pairs of the rows [r0, r0 + ROWS) that need token scores, binned by block.
+// The scatter pass also writes the tile table: CTA c the tiles (block, first
+// pair, pair count) of bins c, c + gridDim.x, ...
 constexpr int kPairRows = 64;
 
 template <bool SCATTER>
 __global__ void __launch_bounds__(NT) pair_bin_kernel(RowMap rm, int64_t rows, const int32_t* __restrict__ blocks,
                                                      int B, int m, int k, int nbins, int* __restrict__ cnt,
                                                      const int* __restrict__ off, int* __restrict__ cursor,
-                                                     uint32_t* __restrict__ pairs) {
+                                                     uint32_t* __restrict__ pairs, int4* __restrict__ tiles) {
   extern __shared__ int sh[];
   int* hist = sh;             // [nbins]
   int* base = sh + nbins;     // [nbins] (scatter only)
@@ -312,6 +314,10 @@ __global__ void __launch_bounds__(NT) pair_bin_kernel(RowMap rm, int64_t rows, c
     base[b] = hist[b] ? off[b] + atomicAdd(&cursor[b], hist[b]) : 0;
     hist[b] = 0;
   }
+  for (int b = blockIdx.x; b < nbins; b += gridDim.x) {
+    const int c = cnt[b], o = off[b], to = off[nbins + b];
+    for (int u = threadIdx.x; 128 * u < c; u += NT) tiles[to + u] = make_int4(b, o + 128 * u, min(128, c - 128 * u), 0);
+  }
   __syncthreads();
   row_pairs([&](int64_t i, int s, int b) {
     const int pos = base[b] + atomicAdd(&hist[b], 1);
@@ -319,11 +325,10 @@ __global__ void __launch_bounds__(NT) pair_bin_kernel(RowMap rm, int64_t rows, c
   });
 }
 
-// Single CTA: offsets of every bin, the tile table (block, first pair,
-// pair count) in tiles of <= 128 pairs, and the tile count.
+// Single CTA: each bin's first pair (off[b]) and first tile (off[nbins + b])
+// in tiles of <= 128 pairs, and the tile count.
 __global__ void __launch_bounds__(1024) pair_scan_kernel(int nbins, const int* __restrict__ cnt, int* __restrict__ off,
-                                                        int* __restrict__ cursor, int4* __restrict__ tiles,
-                                                        int* __restrict__ ntiles) {
+                                                        int* __restrict__ cursor, int* __restrict__ ntiles) {
   __shared__ int s_tmp[1024 / 32 + 1];
   __shared__ int carry_pairs, carry_tiles;
   if (threadIdx.x == 0) { carry_pairs = 0; carry_tiles = 0; }
@@ -336,11 +341,9 @@ __global__ void __launch_bounds__(1024) pair_scan_kernel(int nbins, const int* _
     const int ep = block_exclusive_scan<1024>(c, s_tmp, &tot_p);
     const int et = block_exclusive_scan<1024>(nt, s_tmp, &tot_t);
     if (b < nbins) {
-      const int o = carry_pairs + ep;
-      off[b] = o;
+      off[b] = carry_pairs + ep;
+      off[nbins + b] = carry_tiles + et;
       cursor[b] = 0;
-      for (int u = 0; u < nt; ++u)
-        tiles[carry_tiles + et + u] = make_int4(b, o + 128 * u, min(128, c - 128 * u), 0);
     }
     __syncthreads();
     if (threadIdx.x == 0) { carry_pairs += tot_p; carry_tiles += tot_t; }
@@ -965,9 +968,10 @@ void launch_pair_lists(RowMap rm, int64_t rows, const int32_t* blocks, int B, in
   const size_t smem1 = sizeof(int) * nbins, smem2 = 2 * sizeof(int) * nbins;
   cudaFuncSetAttribute(pair_bin_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem1));
   cudaFuncSetAttribute(pair_bin_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem2));
-  pair_bin_kernel<false><<<grid, NT, smem1, s>>>(rm, rows, blocks, B, m, k, nbins, cnt, nullptr, nullptr, nullptr);
-  pair_scan_kernel<<<1, 1024, 0, s>>>(nbins, cnt, off, cursor, tiles, ntiles);
-  pair_bin_kernel<true><<<grid, NT, smem2, s>>>(rm, rows, blocks, B, m, k, nbins, cnt, off, cursor, pairs);
+  pair_bin_kernel<false><<<grid, NT, smem1, s>>>(rm, rows, blocks, B, m, k, nbins, cnt, nullptr, nullptr, nullptr,
+                                                 nullptr);
+  pair_scan_kernel<<<1, 1024, 0, s>>>(nbins, cnt, off, cursor, ntiles);
+  pair_bin_kernel<true><<<grid, NT, smem2, s>>>(rm, rows, blocks, B, m, k, nbins, cnt, off, cursor, pairs, tiles);
 }
 
 void launch_topk_from_keys(RowMap rm, int64_t rows, const int32_t* blocks, const uint32_t* tkeys, int B,
