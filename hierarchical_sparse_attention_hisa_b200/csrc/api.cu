@@ -172,7 +172,7 @@ void run_select_tokens(const hsa_params* p, int64_t Lq, int64_t Lk, const void* 
       *ok = false;
       return;
     }
-    hsa::launch_topk_from_keys(rm, Lq, blocks, tkeys, p->B, p->m, p->k, indices, s);
+    hsa::launch_topk_from_keys(rm, Lq, blocks, tkeys, p->B, p->m, p->k, indices, s, true);
   } else {
     // CUDA-core scoring: the row's candidates (at most m*B, at most Lk) in shared memory
     if (std::min<int64_t>(int64_t(p->m) * p->B, Lk) > kMaxCandidatesSmem) {

@@ -113,6 +113,10 @@ __global__ void __launch_bounds__(sg_threads<GATHER>(), 1) score_gemm_kernel(con
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base;
+  // the set-up above touches no global memory: under a programmatic
+  // dependent launch it overlaps the previous kernel
+  griddep_wait();
+  griddep_launch();
   const int total = GATHER ? *ta.ntiles : ta.m_tiles * ta.nb_tiles;
   bool dead = false;
 
@@ -202,16 +206,19 @@ __global__ void __launch_bounds__(sg_threads<GATHER>(), 1) score_gemm_kernel(con
     const int gw = warp - 6, c = lane % CPR, rsub = lane / CPR;
     const uint4* qb = reinterpret_cast<const uint4*>(ta.qsrc);
     uint32_t it = 0;
-    auto qrow_of = [&](int tt) -> int {
-      if (tt >= total) return 0;
-      const int4 d = ta.tiles[tt];
+    // a tile's descriptor is fetched two tiles ahead, the query row one ahead
+    const int g = int(gridDim.x);
+    auto desc = [&](int tt) { return tt < total ? ta.tiles[tt] : make_int4(0, 0, 0, 0); };
+    auto qrow_of = [&](const int4& d) -> int {
       const int r = 32 * gw + lane;
       return r < d.z ? int(ta.pairs[d.y + r] / uint32_t(ta.m)) : 0;
     };
-    int qn = qrow_of(blockIdx.x);
+    int qn = qrow_of(desc(blockIdx.x));
+    int4 dn = desc(blockIdx.x + g);
     for (int t = blockIdx.x; t < total && !dead; t += gridDim.x) {
       const int qr = qn;
-      qn = qrow_of(t + gridDim.x);  // one tile ahead
+      qn = qrow_of(dn);
+      dn = desc(t + 2 * g);
       const int s = it % C::NS;
       if (!sg_wait_warp(&empty[s], ((it / C::NS) & 1) ^ 1, dead)) break;
       const uint32_t a_s = smem_u32(sm + s * C::STAGE);
@@ -237,11 +244,23 @@ __global__ void __launch_bounds__(sg_threads<GATHER>(), 1) score_gemm_kernel(con
     uint32_t* sb = stage[quad];
     const int rsub = lane >> 3, ch = lane & 7;
     uint32_t it = 0;
+    // gathered mode: a tile's descriptor is fetched two tiles ahead and this
+    // thread's pair one tile ahead, so neither load waits in the loop
+    const int g = int(gridDim.x);
+    auto desc = [&](int tt) { return tt < total ? ta.tiles[tt] : make_int4(0, 0, 0, 0); };
+    auto pair_off = [&](const int4& d) { return r < d.z ? int64_t(ta.pairs[d.y + r]) * ta.ld : int64_t(-1); };
+    int4 d_next = make_int4(0, 0, 0, 0);
+    int64_t off_next = -1;
+    if (GATHER) {
+      off_next = pair_off(desc(blockIdx.x));
+      d_next = desc(blockIdx.x + g);
+    }
     for (int t = blockIdx.x; t < total && !dead; t += gridDim.x) {
       int64_t off = -1;  // element offset of this thread's row in out, or -1
       if (GATHER) {
-        const int4 d = ta.tiles[t];
-        if (r < d.z) off = int64_t(ta.pairs[d.y + r]) * ta.ld;
+        off = off_next;
+        off_next = pair_off(d_next);
+        d_next = desc(t + 2 * g);
       } else {
         const int mt = t / ta.nb_tiles, nt = t % ta.nb_tiles;
         if (!block_tile_needed(ta, mt, nt, N)) continue;
@@ -292,7 +311,7 @@ bool launch_sg(const CUtensorMap& am, const CUtensorMap& bm, const TileArgs& ta,
   using C = SG<DK, N, NSPLIT>;
   auto kern = score_gemm_kernel<DK, N, NSPLIT, GATHER>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess) return false;
-  kern<<<grid, sg_threads<GATHER>(), C::SMEM, s>>>(am, bm, ta);
+  launch_kernel(true, kern, grid, sg_threads<GATHER>(), C::SMEM, s, am, bm, ta);
   count_launches(1);
   return true;
 }
