@@ -24,12 +24,17 @@
 //                one kind of MMA never holds up the other;
 //   warps 6..21  four softmax warpgroups, warpgroup w owning heads
 //                [w*HP/4, (w+1)*HP/4): thread = TMEM lane = key row of the tile.
-// Softmax runs in the exp2 domain with a per-head running maximum that is
-// only raised (and O^T, l rescaled) when a tile exceeds it by more than 2^8,
-// so the cross-thread max reduction happens on a query's first tile and
-// rarely after; the per-tile check is one hardware barrier reduction. P is
-// rounded to bf16 for the second MMA; accumulation is fp32; O is normalised
-// by one reciprocal of the row sum per head.
+// Softmax runs in the exp2 domain. A launch makes two passes. The first
+// keeps each head's running maximum from the item's first tile (the only
+// cross-thread max reduction) and takes every later tile against it; an item
+// whose weights then grow past 2^24 (a partial row sum above it, or not a
+// number), or whose first tile left a head without a finite maximum, is
+// flagged and not written. The second pass takes the flagged items again
+// with a per-tile check, one hardware barrier reduction, that raises the
+// maximum (and rescales O^T, l) when a tile exceeds it by more than 2^8; it
+// exits at once when nothing was flagged. P is rounded to bf16 for the second
+// MMA; accumulation is fp32; O is normalised by one reciprocal of the row sum
+// per head.
 //
 // A barrier probe in an MMA-issuing thread costs about as much as an MMA when
 // MMAs are queued, so with two stages each issuer waits on one barrier per
@@ -39,6 +44,8 @@
 // Every mbarrier wait is bounded. Within a softmax warpgroup all four warps
 // take the same sequence of named barriers: a failed wait is folded into the
 // next barrier reduction, after which the whole warpgroup leaves together.
+#include <atomic>
+
 #include "kernels.cuh"
 #include "tc.cuh"
 
@@ -47,6 +54,12 @@ namespace hsa {
 __device__ int g_attn_err;     // set when a bounded wait gives up
 __device__ int g_attn_inject;  // test hook: short waits and one lost arrival
 
+// Flagged-item lists of the prefill launches: a ring of slots, one per head
+// group of a call (a slot is reused kRedoSlots groups later), each a count and
+// up to kRedoSlotCap items.
+constexpr int kRedoSlots = 64, kRedoSlotCap = 4096;
+__device__ int g_attn_redo[kRedoSlots * (1 + kRedoSlotCap)];
+
 namespace {
 
 using namespace tc;
@@ -54,7 +67,8 @@ using namespace tc;
 constexpr int TILE = 128;    // kept keys per MMA tile (the M dimension)
 constexpr int NWG = 4;       // softmax warpgroups
 constexpr int NPW = 4;       // producer warps: one kept-index row per lane
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr float kRescaleThreshold = 8.0f;  // log2 units (second pass)
+constexpr float kFlagSum = 16777216.0f;    // 2^24: a larger partial row sum flags the item
 constexpr long long kInjectWaitCycles = 1ll << 21;  // about a millisecond
 
 template <int HP, int DH>
@@ -96,7 +110,10 @@ struct Bars {
 // Each query is cut into items_per_query parts of tiles_per_item 128-key
 // tiles; with one part per query the kernel writes normalised O, otherwise
 // every part w = q * items_per_query + s writes its unnormalised O^T, running
-// maximum and row sum for a later combination.
+// maximum and row sum for a later combination. redo[0] counts the items the
+// first pass flagged, listed in redo[1 .. redo_cap] (an item once per softmax
+// warpgroup that flagged it); the second pass takes them in that order, or
+// every item when the count is above redo_cap.
 struct AttnArgs {
   const uint16_t* Q;
   const int32_t* idx;
@@ -106,6 +123,8 @@ struct AttnArgs {
   int items_per_query, tiles_per_item;
   uint16_t* O;
   float *Opart, *mpart, *lpart;  // [items][H][d], [items][H], [items][H]
+  int* redo;                     // [1 + redo_cap]
+  int redo_cap;
 };
 
 namespace {
@@ -260,7 +279,9 @@ HSA_DEV void tmem_st_cols(uint32_t taddr, const float (&v)[N]) {
   tmem_wait_st();
 }
 
-template <int HP, int DH>
+// VOTE false: the first pass over every item; true: the second pass over
+// the flagged ones (launched in stream order after the first).
+template <int HP, int DH, bool VOTE>
 __global__ void __launch_bounds__(32 * Cfg<HP, DH>::NWARPS, 1) sparse_attn_tc_kernel(
     const uint16_t* __restrict__ K, const uint16_t* __restrict__ V, const AttnArgs a) {
   using C = Cfg<HP, DH>;
@@ -268,7 +289,13 @@ __global__ void __launch_bounds__(32 * Cfg<HP, DH>::NWARPS, 1) sparse_attn_tc_ke
   const int Lk = a.Lk, k = a.k, H = a.H;
   const float scale_log2 = a.scale_log2;
   const int ipq = a.items_per_query, tpi = a.tiles_per_item;
-  const int n_items = a.Lq * ipq;
+  if (VOTE) griddep_wait();  // the first pass has finished its list
+  const int flagged_n = VOTE ? *a.redo : 0;
+  const bool listed = VOTE && flagged_n <= a.redo_cap;  // else every item again
+  const int n_items = listed ? flagged_n : a.Lq * ipq;
+  if (VOTE && flagged_n == 0) return;  // nothing flagged (the whole CTA leaves)
+  // the w-th item of this pass
+  auto item = [&](int w) { return listed ? a.redo[1 + w] : w; };
   constexpr int HH = C::HH;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -325,16 +352,16 @@ __global__ void __launch_bounds__(32 * Cfg<HP, DH>::NWARPS, 1) sparse_attn_tc_ke
     // 128B-swizzled K-major tile, before the swizzle of the chunk
     const uint32_t dbase = (cpk >> 3) * (TILE * 128) + (32 * warp + rsub) * 128;
     const TailScan ts{(k & 3) == 0 && k >= 128, ((k & 3) == 0 && k >= 128) ? k - 128 : 0};
-    int4 pre = blockIdx.x < n_items ? ts.window(idx, blockIdx.x / ipq, k) : make_int4(-1, -1, -1, -1);
+    int4 pre = int(blockIdx.x) < n_items ? ts.window(idx, item(blockIdx.x) / ipq, k) : make_int4(-1, -1, -1, -1);
     const bool inject = *(volatile int*)&g_attn_inject != 0;
     uint32_t g = 0, qn = 0;
-    for (int w = blockIdx.x; w < n_items && !dead; w += gridDim.x, ++qn) {
-      const int q = w / ipq, part = w - q * ipq;
+    for (int wi = blockIdx.x; wi < n_items && !dead; wi += gridDim.x, ++qn) {
+      const int w = item(wi), q = w / ipq, part = w - q * ipq;
       const int32_t* row = idx + int64_t(q) * k;
       const uint4* Kq = reinterpret_cast<const uint4*>(K + int64_t(q) * a.kv_stride * DH);
       const uint4* Vq = reinterpret_cast<const uint4*>(V + int64_t(q) * a.kv_stride * DH);
       const int4 win = pre;
-      if (w + int(gridDim.x) < n_items) pre = ts.window(idx, (w + gridDim.x) / ipq, k);
+      if (wi + int(gridDim.x) < n_items) pre = ts.window(idx, item(wi + gridDim.x) / ipq, k);
       const int last = ts.last_valid(win, row, k, Lk);
       const int t0 = part * tpi;                                  // this item's tiles
       const int nt = max(0, min((last + TILE) / TILE, t0 + tpi) - t0);
@@ -393,7 +420,7 @@ __global__ void __launch_bounds__(32 * Cfg<HP, DH>::NWARPS, 1) sparse_attn_tc_ke
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_bf16(128, HP, false, false);
       uint32_t g = 0, qn = 0;
-      for (int w = blockIdx.x; w < n_items && !dead; w += gridDim.x, ++qn) {
+      for (int wi = blockIdx.x; wi < n_items && !dead; wi += gridDim.x, ++qn) {
         const int qb = qn & 1;
         if (!wait_bar(&bars.qfull[qb], (qn >> 1) & 1, dead)) break;
         const int nt = qinfo[qb][1];
@@ -432,7 +459,7 @@ __global__ void __launch_bounds__(32 * Cfg<HP, DH>::NWARPS, 1) sparse_attn_tc_ke
     if (lane == 0) {
       constexpr uint32_t id_o = idesc_bf16(128, HP, true, true);
       uint32_t g = 0, qn = 0, oq = 0;
-      for (int w = blockIdx.x; w < n_items && !dead; w += gridDim.x, ++qn) {
+      for (int wi = blockIdx.x; wi < n_items && !dead; wi += gridDim.x, ++qn) {
         const int qb = qn & 1;
         if (!wait_bar(&bars.qfull[qb], (qn >> 1) & 1, dead)) break;
         const int nt = qinfo[qb][1];
@@ -485,8 +512,8 @@ __global__ void __launch_bounds__(32 * Cfg<HP, DH>::NWARPS, 1) sparse_attn_tc_ke
     const int h0 = wg * HH;                 // first head of this warpgroup
     const uint32_t lane_addr = uint32_t(quad * 32) << 16;
     uint32_t g = 0, qn = 0, oq = 0;
-    for (int w = blockIdx.x; w < n_items; w += gridDim.x, ++qn) {
-      const int q = w / ipq;
+    for (int wi = blockIdx.x; wi < n_items; wi += gridDim.x, ++qn) {
+      const int w = item(wi), q = w / ipq;
       const int qb = qn & 1;
       const bool okq = wait_all(&bars.qfull[qb], (qn >> 1) & 1, dead);
       if (wg_or(bar_id, !okq || dead)) { dead = true; break; }
@@ -550,8 +577,9 @@ __global__ void __launch_bounds__(32 * Cfg<HP, DH>::NWARPS, 1) sparse_attn_tc_ke
         }
         const bool mine = tmax > kRescaleThreshold || !complete;
         dead = dead || !oks;
-        // (a query's first tile always sets the maxima: no vote needed)
-        if (i == 0 || wg_or(bar_id, mine || dead)) {
+        // (a query's first tile always sets the maxima: no vote needed; the
+        // first pass takes no vote at all)
+        if (i == 0 || (VOTE && wg_or(bar_id, mine || dead))) {
           if (wg_or(bar_id, dead)) { quit = true; break; }
           // raise the running maxima of this warpgroup's heads to cover the tile
 #pragma unroll
@@ -639,7 +667,18 @@ __global__ void __launch_bounds__(32 * Cfg<HP, DH>::NWARPS, 1) sparse_attn_tc_ke
 #pragma unroll
         for (int e = 0; e < NL; ++e) red[wq][h0 + transpose_head<HH>(lane, e)] = lp[e];
       }
-      wg_sync(bar_id);
+      // first pass: a head left without a finite maximum by the first tile,
+      // or a partial row sum above 2^24 (or not a number), flags the item, so
+      // every p of an item not flagged is below 2^24 (the sums hold them
+      // whole); the barrier also publishes the row sums
+      bool flag = r < HH && h0 + r < nh && mh[h0 + r] == -INFINITY;
+#pragma unroll
+      for (int e = 0; e < NL; ++e) flag = flag || !(lp[e] <= kFlagSum);
+      const bool flagged = wg_or(bar_id, !VOTE && flag);
+      if (flagged && r == 0) {
+        const int at = atomicAdd(a.redo, 1);
+        if (at < a.redo_cap) a.redo[1 + at] = w;
+      }
       if (r < HH) {
         const float l = red[0][h0 + r] + red[1][h0 + r] + red[2][h0 + r] + red[3][h0 + r];
         lsum[h0 + r] = l;
@@ -647,7 +686,7 @@ __global__ void __launch_bounds__(32 * Cfg<HP, DH>::NWARPS, 1) sparse_attn_tc_ke
       }
       wg_sync(bar_id);
       const bool oko = wait_all(&bars.ofull[ob], (oq >> 1) & 1, dead);
-      if (oko) {
+      if (oko && !flagged) {
         tc_fence_after();
         float ov[HH];
         tmem_ld_cols<HH>(tmem + lane_addr + 2 * HP + ob * HP + h0, ov);
@@ -689,13 +728,18 @@ __global__ void __launch_bounds__(32 * Cfg<HP, DH>::NWARPS, 1) sparse_attn_tc_ke
 template <int HP, int DH>
 bool launch_hp(const AttnArgs& a, const void* K, const void* V, cudaStream_t s, bool pdl) {
   using C = Cfg<HP, DH>;
-  auto kern = sparse_attn_tc_kernel<HP, DH>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+  auto first = sparse_attn_tc_kernel<HP, DH, false>;
+  auto second = sparse_attn_tc_kernel<HP, DH, true>;
+  if (cudaFuncSetAttribute(first, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess ||
+      cudaFuncSetAttribute(second, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
     return false;
   const int64_t items = int64_t(a.Lq) * a.items_per_query;
   const int grid = int(items < num_sms() ? items : num_sms());
-  launch_kernel(pdl, kern, grid, 32 * C::NWARPS, C::SMEM, s, static_cast<const uint16_t*>(K),
-                static_cast<const uint16_t*>(V), a);
+  const auto Kp = static_cast<const uint16_t*>(K);
+  const auto Vp = static_cast<const uint16_t*>(V);
+  launch_kernel(pdl, first, grid, 32 * C::NWARPS, C::SMEM, s, Kp, Vp, a);
+  // the flagged items again (its CTAs leave at once when there are none)
+  launch_kernel(true, second, grid, 32 * C::NWARPS, C::SMEM, s, Kp, Vp, a);
   return true;
 }
 
@@ -706,12 +750,27 @@ bool launch_group(const AttnArgs& a, const void* K, const void* V, cudaStream_t 
   return launch_hp<64, DH>(a, K, V, s, pdl);
 }
 
-// One launch per group of up to 64 heads.
-bool launch_args(AttnArgs a, int d, const void* K, const void* V, cudaStream_t s, bool pdl) {
+// Two launches (the passes) per group of up to 64 heads. With a list given,
+// group g lists its flagged items at redo + g * redo_stride (counts zeroed
+// by the caller, room for every item); otherwise each group takes the next
+// slot of the ring and zeroes its count first.
+bool launch_args(AttnArgs a, int d, const void* K, const void* V, cudaStream_t s, bool pdl, int* redo,
+                 int64_t redo_stride) {
+  static std::atomic<unsigned> next_slot{0};
+  int* ring = nullptr;
+  if (!redo && cudaGetSymbolAddress(reinterpret_cast<void**>(&ring), g_attn_redo) != cudaSuccess) return false;
   for (int h0 = 0; h0 < a.H; h0 += 64) {
     a.h0 = h0;
     a.nh = a.H - h0 < 64 ? a.H - h0 : 64;
-    count_launches(1);
+    if (redo) {
+      a.redo = redo + (h0 / 64) * redo_stride;
+      a.redo_cap = int(redo_stride - 1);
+    } else {
+      a.redo = ring + (next_slot.fetch_add(1) % kRedoSlots) * (1 + kRedoSlotCap);
+      a.redo_cap = kRedoSlotCap;
+      if (cudaMemsetAsync(a.redo, 0, sizeof(int), s) != cudaSuccess) return false;
+    }
+    count_launches(2);
     const bool ok = d == 128 ? launch_group<128>(a, K, V, s, pdl) : launch_group<64>(a, K, V, s, pdl);
     if (!ok) return false;
   }
@@ -724,9 +783,12 @@ bool tc_attn_supported(int H, int d, int64_t Lq, int64_t Lk) {
   return (d == 128 || d == 64) && H >= 1 && Lq * H < (int64_t(1) << 31) && Lk < (int64_t(1) << 31);
 }
 
+int64_t attn_redo_ints(int64_t items) { return 1 + 4 * items; }
+
 bool launch_sparse_attn_tc(int64_t Lq, const void* Q, const void* K, const void* V, const int32_t* idx,
                            int64_t Lk, int k, int H, int d, float scale, void* O, cudaStream_t s) {
   if (Lq == 0) return true;
+
   AttnArgs a{};
   a.Q = static_cast<const uint16_t*>(Q);
   a.idx = idx; a.Lq = int(Lq); a.Lk = int(Lk); a.k = k; a.H = H;
@@ -735,12 +797,12 @@ bool launch_sparse_attn_tc(int64_t Lq, const void* Q, const void* K, const void*
   a.items_per_query = 1;
   a.tiles_per_item = (k + TILE - 1) / TILE;
   a.O = static_cast<uint16_t*>(O);
-  return launch_args(a, d, K, V, s, false);
+  return launch_args(a, d, K, V, s, false, nullptr, 0);
 }
 
 bool launch_sparse_attn_tc_split(int batch, const void* Q, const void* Kc, const void* Vc, const int32_t* idx,
                                  int64_t capacity, int k, int H, int d, float scale, int parts, float* Opart,
-                                 float* mpart, float* lpart, cudaStream_t s, bool pdl) {
+                                 float* mpart, float* lpart, int* redo, cudaStream_t s, bool pdl) {
   if (batch == 0) return true;
   AttnArgs a{};
   a.Q = static_cast<const uint16_t*>(Q);
@@ -751,7 +813,7 @@ bool launch_sparse_attn_tc_split(int batch, const void* Q, const void* Kc, const
   a.tiles_per_item = ((k + TILE - 1) / TILE + parts - 1) / parts;
   a.O = nullptr;
   a.Opart = Opart; a.mpart = mpart; a.lpart = lpart;
-  return launch_args(a, d, Kc, Vc, s, pdl);
+  return launch_args(a, d, Kc, Vc, s, pdl, redo, attn_redo_ints(int64_t(batch) * parts));
 }
 
 // Host side: whether a bounded wait of this kernel gave up on the current

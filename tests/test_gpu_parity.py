@@ -394,6 +394,27 @@ def test_attention_long_context_chunk_sampled(hsa):
     print("1m chunk max/mean abs err", assert_attn_close(got[rows], ref, "1m chunk"))
 
 
+def test_attention_second_pass_many_rows(hsa):
+    # Rows whose later tiles outgrow the first tile's maximum (by ~8 log2
+    # units a tile) are flagged by the first pass and taken again with the
+    # per-tile rescale; more rows than SMs, every head group's warpgroups
+    # flagging the same rows, flat rows (descending order) and short rows
+    # among them.
+    Lq, Lk, H, d, k = 400, 2048, 64, 128, 1024
+    Q = synth.f32_to_bf16_bits(np.ones((Lq, H, d), np.float32)
+                               * (1.0 + np.arange(H, dtype=np.float32) / 64)[None, :, None])
+    K = synth.f32_to_bf16_bits(np.repeat(0.5 * (np.arange(Lk) // 128), d).reshape(Lk, d).astype(np.float32))
+    V = synth.normal_bf16((Lk, d), 28, 5)
+    rng = np.random.default_rng(28)
+    idx = np.full((Lq, k), -1, dtype=np.int32)
+    for i in range(Lq):
+        n = k if i % 5 else int(rng.integers(1, k + 1))
+        row = np.sort(rng.choice(Lk, size=n, replace=False)).astype(np.int32)
+        idx[i, :n] = row[::-1] if i % 2 else row
+    got = run_attn(hsa, Q, K, V, idx)
+    assert_attn_close(got, oracle.sparse_attn(Q, K, V, idx), "second pass")
+
+
 # ------------------------------------------------------------------ decode
 
 def decode_case(hsa, B, m, k, d_idx, H, d, ctx0, capacity, steps, seed, check_seqs=None):
