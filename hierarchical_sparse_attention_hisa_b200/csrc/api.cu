@@ -312,12 +312,10 @@ namespace {
 // Workspace of a decode step (256-byte aligned regions):
 //   blocks [batch][m] i32, indices [batch][k] i32 (unless the caller takes them),
 //   block-score keys [batch][capacity/B] u32, token-score keys [batch][m*B] u32,
-//   attention parts: O [batch*parts][H][d] f32, maxima and row sums [batch*parts][H] f32,
-//   the attention's flagged-part lists, one per group of 64 heads.
+//   attention parts: O [batch*parts][H][d] f32, maxima and row sums [batch*parts][H] f32.
 struct DecodeWs {
-  size_t blocks, idx, bkeys, tkeys, opart, mpart, lpart, redo, total;
-  int parts, ngroups;
-  int64_t redo_stride;
+  size_t blocks, idx, bkeys, tkeys, opart, mpart, lpart, total;
+  int parts;
 };
 DecodeWs decode_ws(const hsa_params* p, int32_t batch, int64_t capacity) {
   DecodeWs w{};
@@ -334,9 +332,6 @@ DecodeWs decode_ws(const hsa_params* p, int32_t batch, int64_t capacity) {
   w.opart = take(size_t(batch) * w.parts * p->H * p->d * 4);
   w.mpart = take(size_t(batch) * w.parts * p->H * 4);
   w.lpart = take(size_t(batch) * w.parts * p->H * 4);
-  w.ngroups = (p->H + 63) / 64;
-  w.redo_stride = hsa::attn_redo_ints(int64_t(batch) * w.parts);
-  w.redo = take(size_t(w.ngroups) * w.redo_stride * 4);
   w.total = o;
   return w;
 }
@@ -387,10 +382,9 @@ int hsa_decode_step(const hsa_params* p, int32_t batch, int64_t capacity, int32_
   // 1. append the new token (and the block sum of a block it completes), in
   //    the same kernel as 2. the block scores against the block-sum cache;
   //    top-m with the forced blocks
-  int* redo = reinterpret_cast<int*>(ws + w.redo);
   hsa::launch_decode_block_scores(batch, capacity, ctx_len, p->B, p->m, p->d_idx, q_idx_new, ksum_cache,
                                   bkeys, nbc, p->d, k_idx_cache, K_cache, V_cache, ksum_cache, k_idx_new,
-                                  K_new, V_new, redo, w.redo_stride, w.ngroups, stream);
+                                  K_new, V_new, stream);
   hsa::launch_topm_from_keys(rm, batch, bkeys, nbc, p->B, p->m, nbc > 2 ? nbc - 2 : 1, blocks, stream, true);
   // 3. token scores inside the kept blocks, top-k
   hsa::launch_decode_token_scores(batch, capacity, ctx_len, p->B, p->m, p->d_idx, blocks, q_idx_new,
@@ -403,7 +397,7 @@ int hsa_decode_step(const hsa_params* p, int32_t batch, int64_t capacity, int32_
   float* mpart = reinterpret_cast<float*>(ws + w.mpart);
   float* lpart = reinterpret_cast<float*>(ws + w.lpart);
   if (!hsa::launch_sparse_attn_tc_split(batch, Q_new, K_cache, V_cache, idx, capacity, p->k, p->H, p->d,
-                                        softmax_scale(p), w.parts, opart, mpart, lpart, redo, stream, true))
+                                        softmax_scale(p), w.parts, opart, mpart, lpart, stream, true))
     return HSA_ERR_CUDA;
   hsa::launch_decode_combine(batch, capacity, ctx_len, p->H, p->d, w.parts, opart, mpart, lpart, O, stream);
   return launch_status();

@@ -24,15 +24,16 @@
 //                one kind of MMA never holds up the other;
 //   warps 6..21  four softmax warpgroups, warpgroup w owning heads
 //                [w*HP/4, (w+1)*HP/4): thread = TMEM lane = key row of the tile.
-// Softmax runs in the exp2 domain. A launch makes two passes. The first
-// keeps each head's running maximum from the item's first tile (the only
-// cross-thread max reduction) and takes every later tile against it; an item
-// whose weights then grow past 2^24 (a partial row sum above it, or not a
-// number), or whose first tile left a head without a finite maximum, is
-// flagged and not written. The second pass takes the flagged items again
-// with a per-tile check, one hardware barrier reduction, that raises the
-// maximum (and rescales O^T, l) when a tile exceeds it by more than 2^8; it
-// exits at once when nothing was flagged. P is rounded to bf16 for the second
+// Softmax runs in the exp2 domain, in two passes (two launches) for a
+// prefill call. The first keeps each head's running maximum from the item's
+// first tile (the only cross-thread max reduction) and takes every later tile
+// against it; an item whose weights then grow past 2^24 (a partial row sum
+// above it, or not a number), or whose first tile left a head without a
+// finite maximum, is flagged and not written. The second pass takes the
+// flagged items again with a per-tile check, one hardware barrier reduction,
+// that raises the maximum (and rescales O^T, l) when a tile exceeds it by more
+// than 2^8; it exits at once when nothing was flagged. The decode step, whose
+// parts are a few tiles long, runs the second pass alone over every part. P is rounded to bf16 for the second
 // MMA; accumulation is fp32; O is normalised by one reciprocal of the row sum
 // per head.
 //
@@ -113,7 +114,8 @@ struct Bars {
 // maximum and row sum for a later combination. redo[0] counts the items the
 // first pass flagged, listed in redo[1 .. redo_cap] (an item once per softmax
 // warpgroup that flagged it); the second pass takes them in that order, or
-// every item when the count is above redo_cap.
+// every item when the count is above redo_cap or there is no list (a launch
+// of the second pass alone, as the decode step makes).
 struct AttnArgs {
   const uint16_t* Q;
   const int32_t* idx;
@@ -290,10 +292,10 @@ __global__ void __launch_bounds__(32 * Cfg<HP, DH>::NWARPS, 1) sparse_attn_tc_ke
   const float scale_log2 = a.scale_log2;
   const int ipq = a.items_per_query, tpi = a.tiles_per_item;
   if (VOTE) griddep_wait();  // the first pass has finished its list
-  const int flagged_n = VOTE ? *a.redo : 0;
-  const bool listed = VOTE && flagged_n <= a.redo_cap;  // else every item again
+  const int flagged_n = VOTE && a.redo ? *a.redo : 0;
+  const bool listed = VOTE && a.redo && flagged_n <= a.redo_cap;  // else every item
   const int n_items = listed ? flagged_n : a.Lq * ipq;
-  if (VOTE && flagged_n == 0) return;  // nothing flagged (the whole CTA leaves)
+  if (VOTE && a.redo && flagged_n == 0) return;  // nothing flagged (the whole CTA leaves)
   // the w-th item of this pass
   auto item = [&](int w) { return listed ? a.redo[1 + w] : w; };
   constexpr int HH = C::HH;
@@ -725,8 +727,10 @@ __global__ void __launch_bounds__(32 * Cfg<HP, DH>::NWARPS, 1) sparse_attn_tc_ke
 
 // 4 producer warps + 2 MMA-issuing warps + 16 softmax warps = 22 warps (80
 // registers per thread).
+// two_pass: the first pass and then the second over the flagged items;
+// otherwise the second pass alone over every item.
 template <int HP, int DH>
-bool launch_hp(const AttnArgs& a, const void* K, const void* V, cudaStream_t s, bool pdl) {
+bool launch_hp(const AttnArgs& a, const void* K, const void* V, cudaStream_t s, bool pdl, bool two_pass) {
   using C = Cfg<HP, DH>;
   auto first = sparse_attn_tc_kernel<HP, DH, false>;
   auto second = sparse_attn_tc_kernel<HP, DH, true>;
@@ -737,6 +741,10 @@ bool launch_hp(const AttnArgs& a, const void* K, const void* V, cudaStream_t s, 
   const int grid = int(items < num_sms() ? items : num_sms());
   const auto Kp = static_cast<const uint16_t*>(K);
   const auto Vp = static_cast<const uint16_t*>(V);
+  if (!two_pass) {
+    launch_kernel(pdl, second, grid, 32 * C::NWARPS, C::SMEM, s, Kp, Vp, a);
+    return true;
+  }
   launch_kernel(pdl, first, grid, 32 * C::NWARPS, C::SMEM, s, Kp, Vp, a);
   // the flagged items again (its CTAs leave at once when there are none)
   launch_kernel(true, second, grid, 32 * C::NWARPS, C::SMEM, s, Kp, Vp, a);
@@ -744,34 +752,32 @@ bool launch_hp(const AttnArgs& a, const void* K, const void* V, cudaStream_t s, 
 }
 
 template <int DH>
-bool launch_group(const AttnArgs& a, const void* K, const void* V, cudaStream_t s, bool pdl) {
-  if (a.nh <= 16) return launch_hp<16, DH>(a, K, V, s, pdl);
-  if (a.nh <= 32) return launch_hp<32, DH>(a, K, V, s, pdl);
-  return launch_hp<64, DH>(a, K, V, s, pdl);
+bool launch_group(const AttnArgs& a, const void* K, const void* V, cudaStream_t s, bool pdl, bool two_pass) {
+  if (a.nh <= 16) return launch_hp<16, DH>(a, K, V, s, pdl, two_pass);
+  if (a.nh <= 32) return launch_hp<32, DH>(a, K, V, s, pdl, two_pass);
+  return launch_hp<64, DH>(a, K, V, s, pdl, two_pass);
 }
 
-// Two launches (the passes) per group of up to 64 heads. With a list given,
-// group g lists its flagged items at redo + g * redo_stride (counts zeroed
-// by the caller, room for every item); otherwise each group takes the next
-// slot of the ring and zeroes its count first.
-bool launch_args(AttnArgs a, int d, const void* K, const void* V, cudaStream_t s, bool pdl, int* redo,
-                 int64_t redo_stride) {
+// Per group of up to 64 heads: with two_pass, both passes, the group taking
+// the next slot of the ring for its list (count zeroed first); otherwise the
+// second pass alone over every item (one launch).
+bool launch_args(AttnArgs a, int d, const void* K, const void* V, cudaStream_t s, bool pdl, bool two_pass) {
   static std::atomic<unsigned> next_slot{0};
   int* ring = nullptr;
-  if (!redo && cudaGetSymbolAddress(reinterpret_cast<void**>(&ring), g_attn_redo) != cudaSuccess) return false;
+  if (two_pass && cudaGetSymbolAddress(reinterpret_cast<void**>(&ring), g_attn_redo) != cudaSuccess)
+    return false;
   for (int h0 = 0; h0 < a.H; h0 += 64) {
     a.h0 = h0;
     a.nh = a.H - h0 < 64 ? a.H - h0 : 64;
-    if (redo) {
-      a.redo = redo + (h0 / 64) * redo_stride;
-      a.redo_cap = int(redo_stride - 1);
-    } else {
+    a.redo = nullptr;
+    if (two_pass) {
       a.redo = ring + (next_slot.fetch_add(1) % kRedoSlots) * (1 + kRedoSlotCap);
       a.redo_cap = kRedoSlotCap;
       if (cudaMemsetAsync(a.redo, 0, sizeof(int), s) != cudaSuccess) return false;
     }
-    count_launches(2);
-    const bool ok = d == 128 ? launch_group<128>(a, K, V, s, pdl) : launch_group<64>(a, K, V, s, pdl);
+    count_launches(two_pass ? 2 : 1);
+    const bool ok = d == 128 ? launch_group<128>(a, K, V, s, pdl, two_pass)
+                             : launch_group<64>(a, K, V, s, pdl, two_pass);
     if (!ok) return false;
   }
   return true;
@@ -782,8 +788,6 @@ bool launch_args(AttnArgs a, int d, const void* K, const void* V, cudaStream_t s
 bool tc_attn_supported(int H, int d, int64_t Lq, int64_t Lk) {
   return (d == 128 || d == 64) && H >= 1 && Lq * H < (int64_t(1) << 31) && Lk < (int64_t(1) << 31);
 }
-
-int64_t attn_redo_ints(int64_t items) { return 1 + 4 * items; }
 
 bool launch_sparse_attn_tc(int64_t Lq, const void* Q, const void* K, const void* V, const int32_t* idx,
                            int64_t Lk, int k, int H, int d, float scale, void* O, cudaStream_t s) {
@@ -797,12 +801,12 @@ bool launch_sparse_attn_tc(int64_t Lq, const void* Q, const void* K, const void*
   a.items_per_query = 1;
   a.tiles_per_item = (k + TILE - 1) / TILE;
   a.O = static_cast<uint16_t*>(O);
-  return launch_args(a, d, K, V, s, false, nullptr, 0);
+  return launch_args(a, d, K, V, s, false, true);
 }
 
 bool launch_sparse_attn_tc_split(int batch, const void* Q, const void* Kc, const void* Vc, const int32_t* idx,
                                  int64_t capacity, int k, int H, int d, float scale, int parts, float* Opart,
-                                 float* mpart, float* lpart, int* redo, cudaStream_t s, bool pdl) {
+                                 float* mpart, float* lpart, cudaStream_t s, bool pdl) {
   if (batch == 0) return true;
   AttnArgs a{};
   a.Q = static_cast<const uint16_t*>(Q);
@@ -813,7 +817,8 @@ bool launch_sparse_attn_tc_split(int batch, const void* Q, const void* Kc, const
   a.tiles_per_item = ((k + TILE - 1) / TILE + parts - 1) / parts;
   a.O = nullptr;
   a.Opart = Opart; a.mpart = mpart; a.lpart = lpart;
-  return launch_args(a, d, Kc, Vc, s, pdl, redo, attn_redo_ints(int64_t(batch) * parts));
+  // parts of at most a few tiles: the per-tile vote costs less there than a second launch
+  return launch_args(a, d, Kc, Vc, s, pdl, false);
 }
 
 // Host side: whether a bounded wait of this kernel gave up on the current

@@ -50,12 +50,9 @@ __global__ void __launch_bounds__(256) decode_block_scores_kernel(const int32_t*
                                                                   const uint16_t* __restrict__ q_new,
                                                                   const float* __restrict__ ksum_cache,
                                                                   uint32_t* __restrict__ bkeys, int64_t ld,
-                                                                  AppendArgs ap, int* __restrict__ redo,
-                                                                  int64_t redo_stride, int ngroups) {
+                                                                  AppendArgs ap) {
   griddep_wait();
   griddep_launch();
-  // the step's attention lists start empty (the previous step's are done)
-  if (blockIdx.x == 0 && blockIdx.y == 0 && int(threadIdx.x) < ngroups) redo[threadIdx.x * redo_stride] = 0;
   constexpr int VPL = DI / 32;  // fp32 values per lane
   const int64_t b = blockIdx.x;
   const int64_t t = ctx[b];
@@ -205,8 +202,7 @@ __global__ void decode_combine_kernel(int32_t* __restrict__ ctx, int64_t capacit
 void launch_decode_block_scores(int batch, int64_t capacity, const int32_t* ctx, int B, int m, int d_idx,
                                 const void* q_new, const float* ksum_cache, uint32_t* bkeys, int64_t ld,
                                 int d, void* k_idx_cache, void* K_cache, void* V_cache, float* ksum_w,
-                                const void* k_idx_new, const void* K_new, const void* V_new, int* redo,
-                                int64_t redo_stride, int ngroups, cudaStream_t s) {
+                                const void* k_idx_new, const void* K_new, const void* V_new, cudaStream_t s) {
   if (batch == 0) return;
   const int64_t nbmax = capacity / B;
   const int per_cta = 64;
@@ -216,10 +212,10 @@ void launch_decode_block_scores(int batch, int64_t capacity, const int32_t* ctx,
   count_launches(1);
   if (d_idx == 128)
     launch_kernel(true, decode_block_scores_kernel<128>, grid, 256, 0, s, ctx, capacity, B, m, per_cta,
-                  (const uint16_t*)q_new, (const float*)ksum_cache, bkeys, ld, ap, redo, redo_stride, ngroups);
+                  (const uint16_t*)q_new, (const float*)ksum_cache, bkeys, ld, ap);
   else
     launch_kernel(true, decode_block_scores_kernel<64>, grid, 256, 0, s, ctx, capacity, B, m, per_cta,
-                  (const uint16_t*)q_new, (const float*)ksum_cache, bkeys, ld, ap, redo, redo_stride, ngroups);
+                  (const uint16_t*)q_new, (const float*)ksum_cache, bkeys, ld, ap);
 }
 
 void launch_decode_token_scores(int batch, int64_t capacity, const int32_t* ctx, int B, int m, int d_idx,

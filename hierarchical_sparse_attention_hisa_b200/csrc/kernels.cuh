@@ -63,25 +63,19 @@ void launch_pair_lists(RowMap rm, int64_t rows, const int32_t* blocks, int B, in
 void launch_topk_from_keys(RowMap rm, int64_t rows, const int32_t* blocks, const uint32_t* tkeys, int B,
                            int m, int k, int32_t* indices, cudaStream_t s, bool pdl = false);
 // (also appends each sequence's new token: k_idx/K/V rows and a completed block's sum)
-// (also zeroes the counts redo[g * redo_stride], g < ngroups, of the step's attention lists)
 void launch_decode_block_scores(int batch, int64_t capacity, const int32_t* ctx, int B, int m, int d_idx,
                                 const void* q_new, const float* ksum_cache, uint32_t* bkeys, int64_t ld,
                                 int d, void* k_idx_cache, void* K_cache, void* V_cache, float* ksum_w,
-                                const void* k_idx_new, const void* K_new, const void* V_new, int* redo,
-                                int64_t redo_stride, int ngroups, cudaStream_t s);
+                                const void* k_idx_new, const void* K_new, const void* V_new, cudaStream_t s);
 void launch_decode_token_scores(int batch, int64_t capacity, const int32_t* ctx, int B, int m, int d_idx,
                                 const int32_t* blocks, const void* q_new, const void* k_idx_cache,
                                 uint32_t* tkeys, cudaStream_t s);
 // (also advances ctx: every sequence that took the step grows by one token)
 void launch_decode_combine(int batch, int64_t capacity, int32_t* ctx, int H, int d, int parts,
                            const float* Opart, const float* mpart, const float* lpart, void* O, cudaStream_t s);
-// redo: one list per group of 64 heads, attn_redo_ints(batch * parts) ints
-// each, whose counts (the first int) the caller has zeroed in stream order.
 bool launch_sparse_attn_tc_split(int batch, const void* Q, const void* Kc, const void* Vc, const int32_t* idx,
                                  int64_t capacity, int k, int H, int d, float scale, int parts, float* Opart,
-                                 float* mpart, float* lpart, int* redo, cudaStream_t s, bool pdl = false);
-// Ints of one flagged-item list of the attention's two passes over `items` items.
-int64_t attn_redo_ints(int64_t items);
+                                 float* mpart, float* lpart, cudaStream_t s, bool pdl = false);
 
 // Sticky per-device flags set by a bounded wait that gave up (1), read on the
 // host with a synchronous copy and optionally cleared; -1 on a CUDA error.
