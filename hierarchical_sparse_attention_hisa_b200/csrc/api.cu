@@ -145,7 +145,7 @@ void run_select_blocks(const hsa_params* p, int64_t Lq, int64_t Lk, const void* 
       *ok = false;
       return;
     }
-    hsa::launch_topm_from_keys(rm, Lq, bkeys, w.ldb, p->B, p->m, max_block_candidates(p, Lk), blocks, s);
+    hsa::launch_topm_from_keys(rm, Lq, bkeys, w.ldb, p->B, p->m, max_block_candidates(p, Lk), blocks, s, true);
   } else {
     hsa::launch_select_blocks(rm, Lq, q_idx, ksum, 0, p->B, p->m, p->d_idx, blocks,
                               max_block_candidates(p, Lk), s);

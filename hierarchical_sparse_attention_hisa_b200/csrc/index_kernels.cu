@@ -55,6 +55,8 @@ void launch_block_sums(const void* k_idx, int64_t Lk, int B, int d_idx, float* k
 // products are exact and the three partial dot products add up in fp32).
 // ---------------------------------------------------------------------------
 __global__ void ksum_split_kernel(const float* __restrict__ ksum, int64_t n, uint16_t* __restrict__ split) {
+  griddep_wait();
+  griddep_launch();
   for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < n; e += int64_t(gridDim.x) * blockDim.x) {
     const float x = ksum[e];
     const uint32_t hi = f32_to_bf16_rn(x);
@@ -71,7 +73,8 @@ void launch_ksum_split(const float* ksum, int64_t n, void* split, cudaStream_t s
   if (n == 0) return;
   count_launches(1);
   const int64_t blocks = (n + 255) / 256;
-  ksum_split_kernel<<<unsigned(blocks < 4096 ? blocks : 4096), 256, 0, s>>>(ksum, n, (uint16_t*)split);
+  launch_kernel(true, ksum_split_kernel, unsigned(blocks < 4096 ? blocks : 4096), 256, 0, s, ksum, n,
+                (uint16_t*)split);
 }
 
 // ---------------------------------------------------------------------------

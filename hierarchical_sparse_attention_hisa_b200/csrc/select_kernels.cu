@@ -284,6 +284,8 @@ __global__ void __launch_bounds__(NT) pair_bin_kernel(RowMap rm, int64_t rows, c
                                                      int B, int m, int k, int nbins, int* __restrict__ cnt,
                                                      const int* __restrict__ off, int* __restrict__ cursor,
                                                      uint32_t* __restrict__ pairs, int4* __restrict__ tiles) {
+  griddep_wait();
+  griddep_launch();
   extern __shared__ int sh[];
   int* hist = sh;             // [nbins]
   int* base = sh + nbins;     // [nbins] (scatter only)
@@ -329,6 +331,8 @@ __global__ void __launch_bounds__(NT) pair_bin_kernel(RowMap rm, int64_t rows, c
 // in tiles of <= 128 pairs, and the tile count.
 __global__ void __launch_bounds__(1024) pair_scan_kernel(int nbins, const int* __restrict__ cnt, int* __restrict__ off,
                                                         int* __restrict__ cursor, int* __restrict__ ntiles) {
+  griddep_wait();
+  griddep_launch();
   __shared__ int s_tmp[1024 / 32 + 1];
   __shared__ int carry_pairs, carry_tiles;
   if (threadIdx.x == 0) { carry_pairs = 0; carry_tiles = 0; }
@@ -970,8 +974,10 @@ void launch_pair_lists(RowMap rm, int64_t rows, const int32_t* blocks, int B, in
   cudaFuncSetAttribute(pair_bin_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem2));
   pair_bin_kernel<false><<<grid, NT, smem1, s>>>(rm, rows, blocks, B, m, k, nbins, cnt, nullptr, nullptr, nullptr,
                                                  nullptr);
-  pair_scan_kernel<<<1, 1024, 0, s>>>(nbins, cnt, off, cursor, ntiles);
-  pair_bin_kernel<true><<<grid, NT, smem2, s>>>(rm, rows, blocks, B, m, k, nbins, cnt, off, cursor, pairs, tiles);
+  // the scan and the scatter pass overlap their launches with their predecessors
+  launch_kernel(true, pair_scan_kernel, 1, 1024, 0, s, nbins, cnt, off, cursor, ntiles);
+  launch_kernel(true, pair_bin_kernel<true>, grid, NT, smem2, s, rm, rows, blocks, B, m, k, nbins, cnt,
+                static_cast<const int*>(off), cursor, pairs, tiles);
 }
 
 void launch_topk_from_keys(RowMap rm, int64_t rows, const int32_t* blocks, const uint32_t* tkeys, int B,
