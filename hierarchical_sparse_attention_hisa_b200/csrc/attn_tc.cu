@@ -33,9 +33,9 @@
 // flagged items again with a per-tile check, one hardware barrier reduction,
 // that raises the maximum (and rescales O^T, l) when a tile exceeds it by more
 // than 2^8; it exits at once when nothing was flagged. The decode step, whose
-// parts are a few tiles long, runs the second pass alone over every part. P is rounded to bf16 for the second
-// MMA; accumulation is fp32; O is normalised by one reciprocal of the row sum
-// per head.
+// parts are a few tiles long, runs the second pass alone over every part.
+// P is rounded to bf16 for the second MMA; accumulation is fp32; O is
+// normalised by one reciprocal of the row sum per head.
 //
 // A barrier probe in an MMA-issuing thread costs about as much as an MMA when
 // MMAs are queued, so with two stages each issuer waits on one barrier per
