@@ -545,10 +545,21 @@ __global__ void __launch_bounds__(32 * Cfg<HP, DH>::NWARPS, 1) sparse_attn_tc_ke
       for (int h = 0; h < HH; ++h) { lp[h] = 0.f; nm[h] = 0.f; }
       bool complete = false;
       bool quit = false;
+      // (up to 32 heads: the kept index of the next tile is fetched a tile
+      // ahead; with 64 heads the extra register costs more than it hides)
+      constexpr bool kIdxAhead = HP <= 32;
+      int j_next = kIdxAhead && t0 * TILE + r < k ? __ldg(irow + t0 * TILE + r) : -1;
       for (int i = 0; i < nt; ++i, ++g) {
         const int sb = g & 1;
-        const int pos = (t0 + i) * TILE + r;
-        const int j = pos < k ? __ldg(irow + pos) : -1;
+        int j;
+        if constexpr (kIdxAhead) {
+          j = j_next;
+          const int pn = (t0 + i + 1) * TILE + r;
+          if (i + 1 < nt) j_next = pn < k ? __ldg(irow + pn) : -1;
+        } else {
+          const int pos = (t0 + i) * TILE + r;
+          j = pos < k ? __ldg(irow + pos) : -1;
+        }
         const bool valid = j >= 0 && j < Lk;
         const bool oks = wait_all(&bars.sfull[sb], (g >> 1) & 1, dead);
         float x[HH];
