@@ -132,7 +132,12 @@ HSA_API int hsa_index(const hsa_params* p, int64_t Lq, int64_t Lk, const hsa_bf1
  *   Q [Lq][H][d] bf16; K, V [Lk][d] bf16; indices [Lq][k] int32 (entries < 0
  *   are skipped, entries must be < Lk); O [Lq][H][d] bf16, written.
  * fp32 accumulation, O rounded once to bf16. A row without any valid index
- * yields zeros. */
+ * yields zeros. Two kernel launches per group of 64 heads: the second takes
+ * again the rows whose weights outgrew the first's running maxima; the rows
+ * it takes are listed in one of 64 device-side slots, taken in turn by the
+ * calls (and head groups) of the process, so at most 64 head groups may be
+ * in flight at once across streams (a captured CUDA graph keeps the slot of
+ * its capture). */
 HSA_API int hsa_sparse_attn(const hsa_params* p, int64_t Lq, int64_t Lk, const hsa_bf16* Q,
                     const hsa_bf16* K, const hsa_bf16* V, const int32_t* indices, hsa_bf16* O,
                     cudaStream_t stream);
