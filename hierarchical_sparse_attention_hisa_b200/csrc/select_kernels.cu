@@ -277,11 +277,12 @@ __global__ void __launch_bounds__(32 * kTopmWarpsPerCta) topm_warp_rows_kernel(
 // Pairs of the rows [r0, r0 + ROWS) that need token scores, binned by block.
 // The scatter pass also writes the tile table: CTA c the tiles (block, first
 // pair, pair count) of bins c, c + gridDim.x, ...
-constexpr int kPairRows = 64;
+constexpr int kPairRows = 64;  // rows per CTA, fewer when that leaves SMs idle
 
 template <bool SCATTER>
 __global__ void __launch_bounds__(NT) pair_bin_kernel(RowMap rm, int64_t rows, const int32_t* __restrict__ blocks,
-                                                     int B, int m, int k, int nbins, int* __restrict__ cnt,
+                                                     int B, int m, int k, int nbins, int rows_per_cta,
+                                                     int* __restrict__ cnt,
                                                      const int* __restrict__ off, int* __restrict__ cursor,
                                                      uint32_t* __restrict__ pairs, int4* __restrict__ tiles) {
   griddep_wait();
@@ -291,11 +292,11 @@ __global__ void __launch_bounds__(NT) pair_bin_kernel(RowMap rm, int64_t rows, c
   int* base = sh + nbins;     // [nbins] (scatter only)
   for (int b = threadIdx.x; b < nbins; b += NT) hist[b] = 0;
   __syncthreads();
-  const int64_t r0 = int64_t(blockIdx.x) * kPairRows;
+  const int64_t r0 = int64_t(blockIdx.x) * rows_per_cta;
   // one warp per row at a time; lanes over slots
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   auto row_pairs = [&](auto&& fn) {
-    for (int rr = warp; rr < kPairRows; rr += NT / 32) {
+    for (int rr = warp; rr < rows_per_cta; rr += NT / 32) {
       const int64_t i = r0 + rr;
       if (i >= rows) break;
       const int32_t* blk = blocks + i * m;
@@ -968,15 +969,17 @@ void launch_pair_lists(RowMap rm, int64_t rows, const int32_t* blocks, int B, in
   if (rows == 0) return;
   count_launches(3);
   cudaMemsetAsync(cnt, 0, sizeof(int) * nbins, s);
-  const unsigned grid = unsigned((rows + kPairRows - 1) / kPairRows);
+  int rpc = kPairRows;
+  while (rpc > 16 && (rows + rpc - 1) / rpc < 2 * int64_t(num_sms())) rpc /= 2;
+  const unsigned grid = unsigned((rows + rpc - 1) / rpc);
   const size_t smem1 = sizeof(int) * nbins, smem2 = 2 * sizeof(int) * nbins;
   cudaFuncSetAttribute(pair_bin_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem1));
   cudaFuncSetAttribute(pair_bin_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem2));
-  pair_bin_kernel<false><<<grid, NT, smem1, s>>>(rm, rows, blocks, B, m, k, nbins, cnt, nullptr, nullptr, nullptr,
-                                                 nullptr);
+  pair_bin_kernel<false><<<grid, NT, smem1, s>>>(rm, rows, blocks, B, m, k, nbins, rpc, cnt, nullptr, nullptr,
+                                                 nullptr, nullptr);
   // the scan and the scatter pass overlap their launches with their predecessors
   launch_kernel(true, pair_scan_kernel, 1, 1024, 0, s, nbins, cnt, off, cursor, ntiles);
-  launch_kernel(true, pair_bin_kernel<true>, grid, NT, smem2, s, rm, rows, blocks, B, m, k, nbins, cnt,
+  launch_kernel(true, pair_bin_kernel<true>, grid, NT, smem2, s, rm, rows, blocks, B, m, k, nbins, rpc, cnt,
                 static_cast<const int*>(off), cursor, pairs, tiles);
 }
 
